@@ -1,0 +1,362 @@
+"""Benchmark of the routed int4 MoE layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl b200|reference]
+                    [--workload decode|prefill|zipf|tiny] [--no-extra]
+
+One step = one MoE layer (routing, gate/up, down, combine) over one batch of
+synthetic inputs already resident in HBM. The headline workload is the decode
+layer (T=1, H=2048, E=256, top-8, I=Is=512); the prefill (T=512) and uneven
+Zipf (T=4096) layers are measured the same way and reported under "extra".
+Weights rotate over device replicas whose touched bytes exceed 4x the L2, so
+every step reads its weights from HBM.
+
+Multi-GPU: one process per GPU; each rank runs its own batch (tokens are
+independent), no collective on the data path; value = all ranks' tokens over
+the slowest rank's time ("scaling": "weak").
+
+--impl reference times the fp64 CPU oracle on bounded samples of the same
+workload, on the host cores.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from bit_grouped_expert_softmax_b200 import synth  # noqa: E402
+
+METRIC = "MoE-layer tokens/s"
+PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(PEAKS_FALLBACK), "fallback"
+
+
+# ----------------------------------------------------------------------------
+# clocks sampling during the timed region
+# ----------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------
+# workloads
+# ----------------------------------------------------------------------------
+
+def touched_experts(inp):
+    """Distinct routed experts the batch touches (+1 for the shared expert).
+
+    Counted from the logits with a stable argsort, the generator's own view of
+    which experts a token's largest logits select."""
+    order = np.argsort(-inp.logits, axis=1, kind="stable")[:, :inp.k]
+    return len(np.unique(order)) + 1
+
+
+def roofline_numbers(inp, peaks):
+    ex = touched_experts(inp)
+    wbytes = ex * synth.expert_bytes(inp.H, inp.I)
+    flops = synth.layer_flops(inp.T, inp.H, inp.k, inp.I)
+    t_hbm = wbytes / (peaks["hbm_gbs"] * 1e9)
+    t_tc = flops / (peaks["bf16_tflops"] * 1e12)
+    return dict(touched=ex, weight_bytes=wbytes, flops=flops, t_hbm=t_hbm, t_tc=t_tc,
+                bound="hbm" if t_hbm >= t_tc else "tensor")
+
+
+def run_gpu(args, rank, world, local_rank):
+    import torch
+    from bit_grouped_expert_softmax_b200 import api
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    peaks, peaks_kind = load_peaks()
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+
+    def measure(name, steps, warmup):
+        inp = synth.make_workload(name)
+        rf = roofline_numbers(inp, peaks)
+        base = api.DeviceLayer.from_inputs(inp, dev)
+        layer_bytes = sum(t.numel() * t.element_size() for t in base.args())
+        touched = max(rf["weight_bytes"], 1)
+        n_rep = int(min(32, max(2, -(-4 * l2 // touched))))
+        n_rep = int(min(n_rep, max(2, (40 << 30) // layer_bytes)))
+        reps = [base] + [api.DeviceLayer(*[t.clone() for t in base.args()]) for _ in range(n_rep - 1)]
+        x = torch.from_numpy(inp.x.view(np.int16)).to(dev)
+        logits = torch.from_numpy(inp.logits).to(dev)
+        out = torch.empty_like(x)
+        plan = api.Plan(inp.T, inp.H, inp.E, inp.k, inp.I, inp.Is)
+        stream = torch.cuda.current_stream(dev)
+        launches_per_step = 1 if inp.T <= 8 else 6
+
+        def step(i):
+            api.moe_forward(plan.handle, inp.T, x, logits, *reps[i % n_rep].args(), out, stream)
+
+        for i in range(warmup):
+            step(i)
+        plan.status_sync(stream)
+        # CUDA graph of n_rep consecutive steps (one pass over the replicas)
+        graph = None
+        try:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=stream):
+                for i in range(n_rep):
+                    step(i)
+            g.replay()
+            torch.cuda.synchronize(dev)
+            plan.status_sync(stream)
+            graph = g
+        except Exception as e:  # capture unsupported: time eager launches
+            print(f"[bench] graph capture failed ({e}); timing eager launches", file=sys.stderr)
+            torch.cuda.synchronize(dev)
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with ClockSampler(local_rank) as clk:
+            e0.record(stream)
+            if graph is not None:
+                reps_needed = -(-steps // n_rep)
+                for _ in range(reps_needed):
+                    graph.replay()
+                timed_steps = reps_needed * n_rep
+            else:
+                for i in range(steps):
+                    step(i)
+                timed_steps = steps
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+        ms = e0.elapsed_time(e1)
+        plan.status_sync(stream)
+        if world > 1:
+            t = torch.tensor([ms], device=dev)
+            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+            ms = float(t.item())
+        ms_step = ms / timed_steps
+        tokens_s = inp.T * world / (ms_step * 1e-3)
+        # end to end through the host-buffer entry point (pinned host memory)
+        xh = torch.from_numpy(inp.x.view(np.int16)).pin_memory()
+        lh = torch.from_numpy(inp.logits).pin_memory()
+        oh = torch.empty_like(xh).pin_memory()
+        for i in range(3):
+            api.moe_forward_host(plan.handle, inp.T, xh, lh, *reps[i % n_rep].args(), oh, stream)
+        n_e2e = max(10, min(200, steps))
+        torch.cuda.synchronize(dev)
+        t0 = time.perf_counter()
+        for i in range(n_e2e):
+            api.moe_forward_host(plan.handle, inp.T, xh, lh, *reps[i % n_rep].args(), oh, stream)
+        e2e_s = (time.perf_counter() - t0) / n_e2e
+        plan.status_sync(stream)
+        achieved_gbs = rf["weight_bytes"] / (ms_step * 1e-3) / 1e9
+        achieved_tf = rf["flops"] / (ms_step * 1e-3) / 1e12
+        res = dict(workload=name, T=inp.T, ms_per_step=ms_step, tokens_s=tokens_s, rf=rf,
+                   achieved_gbs=achieved_gbs, achieved_tflops=achieved_tf, n_rep=n_rep,
+                   graph=graph is not None, timed_steps=timed_steps, clocks=clk.summary(),
+                   e2e_tokens_s=inp.T * world / e2e_s,
+                   h2d=inp.T * inp.H * 2 + inp.T * inp.E * 4, d2h=inp.T * inp.H * 2,
+                   launches=launches_per_step * timed_steps, inp=inp)
+        del graph
+        plan.close()
+        return res
+
+    main = measure(args.workload, args.steps, args.warmup)
+    extra = {}
+    if not args.no_extra and world == 1:
+        for name in ("prefill", "zipf"):
+            if name != args.workload:
+                r = measure(name, max(10, args.steps // 4), args.warmup)
+                extra[name] = summarize_extra(r, peaks, peaks_kind)
+    return main, extra, peaks, peaks_kind
+
+
+def roofline_obj(r, peaks, peaks_kind):
+    rf = r["rf"]
+    if rf["bound"] == "hbm":
+        a, p, unit = r["achieved_gbs"], peaks["hbm_gbs"], "GB/s"
+    else:
+        a, p, unit = r["achieved_tflops"], peaks["bf16_tflops"], "TFLOP/s"
+    return {"bound": rf["bound"], "achieved": round(a, 2), "peak": p, "unit": unit, "frac": round(a / p, 4),
+            "traffic": None, "peak_source": peaks_kind,
+            "algorithmic": {"weight_bytes": rf["weight_bytes"], "flops": rf["flops"],
+                            "touched_experts_incl_shared": rf["touched"]},
+            "kernel": "whole layer step (all kernels)"}
+
+
+def summarize_extra(r, peaks, peaks_kind):
+    return {"T": r["T"], "tokens_s": round(r["tokens_s"], 1), "ms_per_step": round(r["ms_per_step"], 5),
+            "effective_tflops": round(r["achieved_tflops"], 2), "achieved_weight_gbs": round(r["achieved_gbs"], 1),
+            "roofline": roofline_obj(r, peaks, peaks_kind), "graph": r["graph"], "clocks": r["clocks"],
+            "e2e_tokens_s": round(r["e2e_tokens_s"], 1)}
+
+
+def cpu_baseline(name, budget_s=15.0):
+    """fp64 oracle on a bounded sample of the workload's tokens, on the host cores."""
+    import oracle
+    inp = synth.make_workload(name)
+    cores = oracle.max_threads()
+    n = min(inp.T, max(1, cores))
+    t0 = time.perf_counter()
+    oracle.moe_forward(inp, x=inp.x[:n], logits=inp.logits[:n])
+    dt = time.perf_counter() - t0
+    per_tok = dt / n
+    n2 = int(min(inp.T if inp.T > 1 else 10 ** 9, max(n, budget_s / per_tok)))
+    xs = np.resize(inp.x, (n2, inp.H)) if n2 > inp.T else inp.x[:n2]
+    ls = np.resize(inp.logits, (n2, inp.E)) if n2 > inp.T else inp.logits[:n2]
+    t0 = time.perf_counter()
+    oracle.moe_forward(inp, x=np.ascontiguousarray(xs), logits=np.ascontiguousarray(ls))
+    dt = time.perf_counter() - t0
+    return {"value": round(n2 / dt, 3), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{n2} tokens of the {name} layer (token rows repeated if T is smaller), fp64, "
+                      f"{dt:.1f} s wall"}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
+    ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "zipf", "tiny"])
+    ap.add_argument("--no-extra", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    wl = synth.WORKLOADS[args.workload]
+    config = {"workload": f"{wl.name}: T={wl.T} H={wl.H} E={wl.E} top_k={wl.k} I={wl.I} Is={wl.Is}, "
+                          f"int4 g64 affine weights, seed {wl.seed}",
+              "T": wl.T, "H": wl.H, "E": wl.E, "top_k": wl.k, "I": wl.I, "Is": wl.Is,
+              "tokens_per_rank": wl.T, "parallelism": f"token-dp{args.gpus}"}
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        import oracle
+        steps = []
+        inp = synth.make_workload(args.workload)
+        n = min(inp.T, max(1, oracle.max_threads()))
+        xs, ls = inp.x[:n], inp.logits[:n]
+        if inp.T < n:
+            xs, ls = np.resize(inp.x, (n, inp.H)), np.resize(inp.logits, (n, inp.E))
+        for i in range(args.warmup + args.steps):
+            t0 = time.perf_counter()
+            oracle.moe_forward(inp, x=np.ascontiguousarray(xs), logits=np.ascontiguousarray(ls))
+            if i >= args.warmup:
+                steps.append(time.perf_counter() - t0)
+        tot = sum(steps)
+        val = n * len(steps) / tot
+        line = {"impl": "reference", "metric": METRIC, "value": round(val, 3), "unit": "tokens/s",
+                "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": round(1e3 * tot / len(steps), 3), "higher_is_better": True, "scaling": "weak",
+                "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config,
+                "cpu_baseline": {"kind": "oracle", "cores": oracle.max_threads(), "value": round(val, 3),
+                                 "unit": "tokens/s",
+                                 "sample": f"{n} tokens of the {args.workload} layer per step"},
+                "e2e": {"value": round(val, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}}
+        print(json.dumps(line))
+        return
+
+    if world > 1:
+        import torch
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    main_r, extra, peaks, peaks_kind = run_gpu(args, rank, world, local_rank)
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(args.workload)
+    if rank == 0:
+        r = main_r
+        line = {"metric": METRIC, "value": round(r["tokens_s"], 1), "unit": "tokens/s", "n_gpus": args.gpus,
+                "steps": r["timed_steps"], "warmup": args.warmup, "ms_per_step": round(r["ms_per_step"], 6),
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+                "data": "synthetic", "config": dict(config, l2=(
+                    f"weights rotate over {r['n_rep']} device replicas "
+                    f"({r['n_rep']} x {r['rf']['weight_bytes'] / 1e6:.1f} MB touched > 4 x L2)"),
+                    graph=r["graph"]),
+                "roofline": roofline_obj(r, peaks, peaks_kind),
+                "effective_tflops": round(r["achieved_tflops"], 3),
+                "cpu_baseline": cpu,
+                "e2e": {"value": round(r["e2e_tokens_s"], 1), "unit": "tokens/s",
+                        "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
+                "gpu_launches": r["launches"], "clocks": r["clocks"], "extra": extra}
+        print(json.dumps(line))
+    if world > 1:
+        import torch
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

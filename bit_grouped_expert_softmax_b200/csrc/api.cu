@@ -1,0 +1,418 @@
+// api.cu -- the C ABI declared in include/moe_b200.h.
+//
+// A plan holds the problem sizes and one device allocation carved into the
+// workspace buffers. Every call validates its arguments on the host, then
+// enqueues kernels on the caller's stream without synchronising.
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "../../include/moe_b200.h"
+#include "kernels.cuh"
+
+namespace moe {
+size_t small_t_smem_bytes(int T, int H, int k, int I, int Is);
+}
+
+using namespace moe;
+
+namespace {
+
+thread_local std::string g_last_error;
+
+moe_status fail(moe_status st, const char *fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+moe_status cuda_fail(cudaError_t err, const char *what) {
+  return fail(MOE_ERR_CUDA, "%s: %s (%s)", what, cudaGetErrorName(err), cudaGetErrorString(err));
+}
+
+#define MOE_CUDA(call, what)                       \
+  do {                                             \
+    cudaError_t err__ = (call);                    \
+    if (err__ != cudaSuccess) return cuda_fail(err__, what); \
+  } while (0)
+
+constexpr size_t kAlign = 256;
+size_t align_up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+// Upper bounds of the two work lists for T tokens.
+int64_t max_gu_items(int64_t T, int64_t E, int64_t k, int64_t I, int64_t Is) {
+  const int64_t R = T * k;
+  return (cdiv(R, kTileN) + std::min<int64_t>(E, R)) * (I / kTileM) + cdiv(T, kTileN) * (Is / kTileM);
+}
+int64_t max_dn_items(int64_t T, int64_t E, int64_t k, int64_t H) {
+  const int64_t R = T * k;
+  return (cdiv(R, kTileN) + std::min<int64_t>(E, R) + cdiv(T, kTileN)) * (H / kTileM);
+}
+
+}  // namespace
+
+struct moe_plan_s {
+  int T_max, H, E, k, I, Is, flags;
+  int device, num_sms;
+  size_t ws_bytes;
+  char *ws;
+  // workspace views
+  int32_t *ids;
+  float *wts;
+  int32_t *xexp;
+  int32_t *chunk;
+  int32_t *offsets;
+  int32_t *perm;
+  int32_t *inv;
+  WorkItem *gu_items;
+  WorkItem *dn_items;
+  int32_t *item_counts;
+  __half *xt;
+  __half *h;
+  __half *y;
+  float *hsmall;
+  DevStatus *status;
+  uint32_t *barrier;
+  uint16_t *x_stage;
+  float *logits_stage;
+  uint16_t *out_stage;
+  int64_t max_gu, max_dn;
+};
+
+namespace {
+
+moe_status check_dims(int T_max, int H, int E, int k, int I, int Is) {
+  if (T_max < 1 || T_max > (1 << 20)) return fail(MOE_ERR_INVALID_ARG, "T_max=%d must be in [1, 2^20]", T_max);
+  if (H < kTileM || H % kTileM) return fail(MOE_ERR_INVALID_ARG, "hidden=%d must be a positive multiple of %d", H, kTileM);
+  if (H > 16384) return fail(MOE_ERR_INVALID_ARG, "hidden=%d exceeds 16384", H);
+  if (I < kTileM || I % kTileM) return fail(MOE_ERR_INVALID_ARG, "inter=%d must be a positive multiple of %d", I, kTileM);
+  if (Is < kTileM || Is % kTileM)
+    return fail(MOE_ERR_INVALID_ARG, "shared_inter=%d must be a positive multiple of %d", Is, kTileM);
+  if (I > 8192 || Is > 8192) return fail(MOE_ERR_INVALID_ARG, "inter sizes above 8192 are not supported");
+  if (E < 1 || E > kMaxExperts) return fail(MOE_ERR_INVALID_ARG, "n_experts=%d must be in [1, %d]", E, kMaxExperts);
+  if (k < 1 || k > E || k > kMaxTopK) return fail(MOE_ERR_INVALID_ARG, "top_k=%d must be in [1, min(E, %d)]", k, kMaxTopK);
+  const int64_t rows = static_cast<int64_t>(T_max) * (k + 1);
+  if (rows * H > (int64_t(1) << 31)) return fail(MOE_ERR_INVALID_ARG, "T_max*(top_k+1)*hidden too large");
+  return MOE_OK;
+}
+
+moe_status check_weights(const moe_plan_s *p, const void *packed, const void *scales, const void *biases,
+                         const void *spacked, const void *sscales, const void *sbiases) {
+  const void *ptrs[6] = {packed, scales, biases, spacked, sscales, sbiases};
+  const char *names[6] = {"packed_w", "scales", "biases", "shared_packed_w", "shared_scales", "shared_biases"};
+  for (int i = 0; i < 6; ++i) {
+    if (!ptrs[i]) return fail(MOE_ERR_INVALID_ARG, "%s is NULL", names[i]);
+    if (!aligned16(ptrs[i])) return fail(MOE_ERR_INVALID_ARG, "%s is not 16-byte aligned", names[i]);
+  }
+  (void)p;
+  return MOE_OK;
+}
+
+bool use_small_t(const moe_plan_s *p, int T) {
+  if (p->flags & MOE_FLAG_FORCE_GROUPED) return false;
+  if (T > kSmallT) return false;
+  return small_t_smem_bytes(T, p->H, p->k, p->I, p->Is) <= 200 * 1024;
+}
+
+LayerWeights make_weights(const void *packed, const void *scales, const void *biases, const void *spacked,
+                          const void *sscales, const void *sbiases) {
+  LayerWeights w;
+  w.packed = static_cast<const uint32_t *>(packed);
+  w.scales = static_cast<const uint16_t *>(scales);
+  w.biases = static_cast<const uint16_t *>(biases);
+  w.sh_packed = static_cast<const uint32_t *>(spacked);
+  w.sh_scales = static_cast<const uint16_t *>(sscales);
+  w.sh_biases = static_cast<const uint16_t *>(sbiases);
+  return w;
+}
+
+// routing kernels: ids/weights, histogram + scan + work lists, scatter (+ gather if x)
+moe_status enqueue_routing(moe_plan_s *p, int T, const float *logits, const uint16_t *x, cudaStream_t s) {
+  const int nchunk = static_cast<int>(cdiv(T, kRouteChunk));
+  route_topk_kernel<<<nchunk, 256, 0, s>>>(T, p->E, p->k, logits, p->ids, p->wts, p->chunk);
+  MOE_CUDA(cudaGetLastError(), "route_topk launch");
+  RouteScanArgs sa;
+  sa.T = T; sa.E = p->E; sa.k = p->k; sa.H = p->H; sa.I = p->I; sa.Is = p->Is; sa.nchunk = nchunk;
+  sa.chunk_cnt = p->chunk; sa.offsets = p->offsets;
+  sa.gu_items = p->gu_items; sa.max_gu = static_cast<int>(p->max_gu);
+  sa.dn_items = p->dn_items; sa.max_dn = static_cast<int>(p->max_dn);
+  sa.item_counts = p->item_counts; sa.status = p->status;
+  route_scan_kernel<<<1, 1024, 0, s>>>(sa);
+  MOE_CUDA(cudaGetLastError(), "route_scan launch");
+  RouteScatterArgs ca;
+  ca.T = T; ca.E = p->E; ca.k = p->k; ca.H = p->H;
+  ca.ids = p->ids; ca.chunk_base = p->chunk; ca.perm = p->perm; ca.inv = p->inv;
+  ca.x = x; ca.xt = p->xt; ca.xexp = p->xexp; ca.status = p->status;
+  route_scatter_kernel<<<nchunk, 256, 0, s>>>(ca);
+  MOE_CUDA(cudaGetLastError(), "route_scatter launch");
+  return MOE_OK;
+}
+
+moe_status enqueue_layer(moe_plan_s *p, int T, const uint16_t *x, const float *logits, const LayerWeights &w,
+                         const uint16_t *residual, uint16_t *out, cudaStream_t s) {
+  if (T == 0) return MOE_OK;
+  if (use_small_t(p, T) || (p->flags & MOE_FLAG_FORCE_SMALL_T)) {
+    if (T > kSmallT || small_t_smem_bytes(T, p->H, p->k, p->I, p->Is) > 200 * 1024)
+      return fail(MOE_ERR_UNSUPPORTED, "small-T path needs T <= %d and a small enough layer", kSmallT);
+    SmallTArgs a;
+    a.T = T; a.E = p->E; a.k = p->k; a.H = p->H; a.I = p->I; a.Is = p->Is;
+    a.x = x; a.logits = logits; a.w = w; a.hbuf = p->hsmall; a.barrier = p->barrier;
+    a.residual = residual; a.out = out; a.status = p->status;
+    MOE_CUDA(launch_small_t(a, p->num_sms, s), "small-T kernel launch");
+    return MOE_OK;
+  }
+  moe_status st = enqueue_routing(p, T, logits, x, s);
+  if (st != MOE_OK) return st;
+  GemmArgs g;
+  g.T = T; g.E = p->E; g.k = p->k; g.H = p->H; g.I = p->I; g.Is = p->Is; g.R = T * p->k;
+  g.w = w; g.xt = p->xt; g.h = p->h;
+  g.h_shared_off = static_cast<int64_t>(p->T_max) * p->k * p->I;
+  g.y = p->y; g.perm = p->perm; g.wts = p->wts; g.xexp = p->xexp; g.status = p->status;
+  g.items = p->gu_items;
+  g.item_count = p->item_counts;
+  g.max_items = static_cast<int>(max_gu_items(T, p->E, p->k, p->I, p->Is));
+  MOE_CUDA(launch_gemm_gate_up(g, p->num_sms, s), "gate/up GEMM launch");
+  g.items = p->dn_items;
+  g.item_count = p->item_counts + 1;
+  g.max_items = static_cast<int>(max_dn_items(T, p->E, p->k, p->H));
+  MOE_CUDA(launch_gemm_down(g, p->num_sms, s), "down GEMM launch");
+  CombineArgs c;
+  c.T = T; c.k = p->k; c.H = p->H; c.R = T * p->k;
+  c.inv = p->inv; c.y = p->y; c.xexp = p->xexp; c.residual = residual; c.out = out;
+  MOE_CUDA(launch_combine(c, s), "combine launch");
+  return MOE_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char *moe_last_error(void) { return g_last_error.c_str(); }
+
+const char *moe_version(void) { return "moe_b200 0.1 (sm_100a)"; }
+
+moe_status moe_plan(int T_max, int hidden, int n_experts, int top_k, int inter, int shared_inter, int flags,
+                    moe_plan_t **out) {
+  g_last_error.clear();
+  if (!out) return fail(MOE_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  moe_status st = check_dims(T_max, hidden, n_experts, top_k, inter, shared_inter);
+  if (st != MOE_OK) return st;
+  if ((flags & MOE_FLAG_FORCE_GROUPED) && (flags & MOE_FLAG_FORCE_SMALL_T))
+    return fail(MOE_ERR_INVALID_ARG, "flags FORCE_GROUPED and FORCE_SMALL_T exclude each other");
+  if (flags & ~(MOE_FLAG_FORCE_GROUPED | MOE_FLAG_FORCE_SMALL_T))
+    return fail(MOE_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
+  int dev = 0, ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || ndev == 0) {
+    cudaGetLastError();
+    return fail(MOE_ERR_NO_DEVICE, "no CUDA device is visible");
+  }
+  MOE_CUDA(cudaGetDevice(&dev), "cudaGetDevice");
+  cudaDeviceProp prop;
+  MOE_CUDA(cudaGetDeviceProperties(&prop, dev), "cudaGetDeviceProperties");
+  if (prop.major != 10 || prop.minor != 0)
+    return fail(MOE_ERR_UNSUPPORTED, "device %d is sm_%d%d; this library is built for sm_100a", dev, prop.major,
+                prop.minor);
+
+  moe_plan_s *p = new moe_plan_s();
+  p->T_max = T_max; p->H = hidden; p->E = n_experts; p->k = top_k; p->I = inter; p->Is = shared_inter;
+  p->flags = flags; p->device = dev; p->num_sms = prop.multiProcessorCount;
+  p->max_gu = max_gu_items(T_max, n_experts, top_k, inter, shared_inter);
+  p->max_dn = max_dn_items(T_max, n_experts, top_k, hidden);
+  const size_t T = T_max, H = hidden, E = n_experts, k = top_k, I = inter, Is = shared_inter;
+  const size_t R = T * k, nchunk = (T + kRouteChunk - 1) / kRouteChunk;
+  const size_t sizes[] = {
+      R * 4,                                 // ids
+      R * 4,                                 // wts
+      T * 4,                                 // xexp
+      nchunk * E * 4,                        // chunk
+      (E + 1) * 4,                           // offsets
+      R * 4,                                 // perm
+      R * 4,                                 // inv
+      static_cast<size_t>(p->max_gu) * sizeof(WorkItem),
+      static_cast<size_t>(p->max_dn) * sizeof(WorkItem),
+      16,                                    // item counts
+      (R + T) * H * 2,                       // xt
+      (R * I + T * Is) * 2,                  // h
+      (R + T) * H * 2,                       // y
+      static_cast<size_t>(kSmallT) * (k + 1) * std::max(I, Is) * 4,  // small-T h
+      sizeof(DevStatus),                     // status
+      16,                                    // barrier
+      T * H * 2,                             // x staging
+      T * E * 4,                             // logits staging
+      T * H * 2,                             // out staging
+  };
+  constexpr int nbuf = sizeof(sizes) / sizeof(sizes[0]);
+  size_t offs[nbuf], total = 0;
+  for (int i = 0; i < nbuf; ++i) {
+    offs[i] = total;
+    total += align_up(sizes[i]);
+  }
+  cudaError_t err = cudaMalloc(&p->ws, total);
+  if (err != cudaSuccess) {
+    delete p;
+    return cuda_fail(err, "workspace cudaMalloc");
+  }
+  p->ws_bytes = total;
+  char *b = p->ws;
+  int i = 0;
+  p->ids = reinterpret_cast<int32_t *>(b + offs[i++]);
+  p->wts = reinterpret_cast<float *>(b + offs[i++]);
+  p->xexp = reinterpret_cast<int32_t *>(b + offs[i++]);
+  p->chunk = reinterpret_cast<int32_t *>(b + offs[i++]);
+  p->offsets = reinterpret_cast<int32_t *>(b + offs[i++]);
+  p->perm = reinterpret_cast<int32_t *>(b + offs[i++]);
+  p->inv = reinterpret_cast<int32_t *>(b + offs[i++]);
+  p->gu_items = reinterpret_cast<WorkItem *>(b + offs[i++]);
+  p->dn_items = reinterpret_cast<WorkItem *>(b + offs[i++]);
+  p->item_counts = reinterpret_cast<int32_t *>(b + offs[i++]);
+  p->xt = reinterpret_cast<__half *>(b + offs[i++]);
+  p->h = reinterpret_cast<__half *>(b + offs[i++]);
+  p->y = reinterpret_cast<__half *>(b + offs[i++]);
+  p->hsmall = reinterpret_cast<float *>(b + offs[i++]);
+  p->status = reinterpret_cast<DevStatus *>(b + offs[i++]);
+  p->barrier = reinterpret_cast<uint32_t *>(b + offs[i++]);
+  p->x_stage = reinterpret_cast<uint16_t *>(b + offs[i++]);
+  p->logits_stage = reinterpret_cast<float *>(b + offs[i++]);
+  p->out_stage = reinterpret_cast<uint16_t *>(b + offs[i++]);
+  err = cudaMemset(p->ws, 0, total);
+  if (err == cudaSuccess) err = cudaDeviceSynchronize();
+  if (err != cudaSuccess) {
+    cudaFree(p->ws);
+    delete p;
+    return cuda_fail(err, "workspace clear");
+  }
+  *out = p;
+  return MOE_OK;
+}
+
+moe_status moe_plan_destroy(moe_plan_t *plan) {
+  g_last_error.clear();
+  if (!plan) return fail(MOE_ERR_INVALID_ARG, "plan is NULL");
+  cudaError_t err = cudaDeviceSynchronize();
+  cudaError_t err2 = cudaFree(plan->ws);
+  delete plan;
+  if (err != cudaSuccess) return cuda_fail(err, "synchronize before free");
+  if (err2 != cudaSuccess) return cuda_fail(err2, "workspace cudaFree");
+  return MOE_OK;
+}
+
+int64_t moe_plan_workspace_bytes(const moe_plan_t *plan) { return plan ? static_cast<int64_t>(plan->ws_bytes) : -1; }
+
+moe_status moe_forward(moe_plan_t *plan, int T, const void *x_bf16, const float *router_logits,
+                       const uint32_t *packed_w, const void *scales, const void *biases,
+                       const uint32_t *shared_packed_w, const void *shared_scales, const void *shared_biases,
+                       void *out_bf16, moe_stream_t stream) {
+  g_last_error.clear();
+  if (!plan) return fail(MOE_ERR_INVALID_ARG, "plan is NULL");
+  if (T < 0 || T > plan->T_max) return fail(MOE_ERR_INVALID_ARG, "T=%d outside [0, T_max=%d]", T, plan->T_max);
+  if (T == 0) return MOE_OK;
+  if (!x_bf16 || !router_logits || !out_bf16) return fail(MOE_ERR_INVALID_ARG, "x, logits and out must not be NULL");
+  if (!aligned16(x_bf16) || !aligned16(router_logits) || !aligned16(out_bf16))
+    return fail(MOE_ERR_INVALID_ARG, "x, logits and out must be 16-byte aligned");
+  if (x_bf16 == out_bf16) return fail(MOE_ERR_INVALID_ARG, "out must not alias x (use moe_stack_forward)");
+  moe_status st = check_weights(plan, packed_w, scales, biases, shared_packed_w, shared_scales, shared_biases);
+  if (st != MOE_OK) return st;
+  const LayerWeights w = make_weights(packed_w, scales, biases, shared_packed_w, shared_scales, shared_biases);
+  return enqueue_layer(plan, T, static_cast<const uint16_t *>(x_bf16), router_logits, w, nullptr,
+                       static_cast<uint16_t *>(out_bf16), reinterpret_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_forward_host(moe_plan_t *plan, int T, const void *x_bf16_host, const float *router_logits_host,
+                            const uint32_t *packed_w, const void *scales, const void *biases,
+                            const uint32_t *shared_packed_w, const void *shared_scales, const void *shared_biases,
+                            void *out_bf16_host, moe_stream_t stream) {
+  g_last_error.clear();
+  if (!plan) return fail(MOE_ERR_INVALID_ARG, "plan is NULL");
+  if (T < 0 || T > plan->T_max) return fail(MOE_ERR_INVALID_ARG, "T=%d outside [0, T_max=%d]", T, plan->T_max);
+  if (T == 0) return MOE_OK;
+  if (!x_bf16_host || !router_logits_host || !out_bf16_host)
+    return fail(MOE_ERR_INVALID_ARG, "host x, logits and out must not be NULL");
+  moe_status st = check_weights(plan, packed_w, scales, biases, shared_packed_w, shared_scales, shared_biases);
+  if (st != MOE_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const size_t xb = static_cast<size_t>(T) * plan->H * 2, lb = static_cast<size_t>(T) * plan->E * 4;
+  MOE_CUDA(cudaMemcpyAsync(plan->x_stage, x_bf16_host, xb, cudaMemcpyHostToDevice, s), "copy x to device");
+  MOE_CUDA(cudaMemcpyAsync(plan->logits_stage, router_logits_host, lb, cudaMemcpyHostToDevice, s),
+           "copy logits to device");
+  const LayerWeights w = make_weights(packed_w, scales, biases, shared_packed_w, shared_scales, shared_biases);
+  st = enqueue_layer(plan, T, plan->x_stage, plan->logits_stage, w, nullptr, plan->out_stage, s);
+  if (st != MOE_OK) return st;
+  MOE_CUDA(cudaMemcpyAsync(out_bf16_host, plan->out_stage, xb, cudaMemcpyDeviceToHost, s), "copy out to host");
+  MOE_CUDA(cudaStreamSynchronize(s), "stream synchronize");
+  return MOE_OK;
+}
+
+moe_status moe_stack_forward(moe_plan_t *plan, int n_layers, int T, void *x_inout_bf16, const float *logits,
+                             const moe_layer_weights *layers, moe_stream_t stream) {
+  g_last_error.clear();
+  if (!plan) return fail(MOE_ERR_INVALID_ARG, "plan is NULL");
+  if (n_layers < 0) return fail(MOE_ERR_INVALID_ARG, "n_layers=%d is negative", n_layers);
+  if (T < 0 || T > plan->T_max) return fail(MOE_ERR_INVALID_ARG, "T=%d outside [0, T_max=%d]", T, plan->T_max);
+  if (T == 0 || n_layers == 0) return MOE_OK;
+  if (!x_inout_bf16 || !logits || !layers) return fail(MOE_ERR_INVALID_ARG, "x, logits and layers must not be NULL");
+  if (!aligned16(x_inout_bf16) || !aligned16(logits)) return fail(MOE_ERR_INVALID_ARG, "x and logits must be 16-byte aligned");
+  for (int l = 0; l < n_layers; ++l) {
+    const moe_layer_weights &L = layers[l];
+    moe_status st = check_weights(plan, L.packed_w, L.scales, L.biases, L.shared_packed_w, L.shared_scales,
+                                  L.shared_biases);
+    if (st != MOE_OK) return fail(st, "layer %d: %s", l, g_last_error.c_str());
+  }
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint16_t *x = static_cast<uint16_t *>(x_inout_bf16);
+  for (int l = 0; l < n_layers; ++l) {
+    const moe_layer_weights &L = layers[l];
+    const LayerWeights w =
+        make_weights(L.packed_w, L.scales, L.biases, L.shared_packed_w, L.shared_scales, L.shared_biases);
+    moe_status st = enqueue_layer(plan, T, x, logits + static_cast<size_t>(l) * T * plan->E, w, x, x, s);
+    if (st != MOE_OK) return st;
+  }
+  return MOE_OK;
+}
+
+moe_status moe_route(moe_plan_t *plan, int T, const float *logits, int32_t *ids, float *w, int32_t *offsets,
+                     int32_t *perm, moe_stream_t stream) {
+  g_last_error.clear();
+  if (!plan) return fail(MOE_ERR_INVALID_ARG, "plan is NULL");
+  if (T < 0 || T > plan->T_max) return fail(MOE_ERR_INVALID_ARG, "T=%d outside [0, T_max=%d]", T, plan->T_max);
+  if (T == 0) return MOE_OK;
+  if (!logits) return fail(MOE_ERR_INVALID_ARG, "logits is NULL");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  moe_status st = enqueue_routing(plan, T, logits, nullptr, s);
+  if (st != MOE_OK) return st;
+  const size_t R = static_cast<size_t>(T) * plan->k;
+  if (ids) MOE_CUDA(cudaMemcpyAsync(ids, plan->ids, R * 4, cudaMemcpyDeviceToDevice, s), "copy ids");
+  if (w) MOE_CUDA(cudaMemcpyAsync(w, plan->wts, R * 4, cudaMemcpyDeviceToDevice, s), "copy w");
+  if (offsets)
+    MOE_CUDA(cudaMemcpyAsync(offsets, plan->offsets, (plan->E + 1) * 4, cudaMemcpyDeviceToDevice, s), "copy offsets");
+  if (perm) MOE_CUDA(cudaMemcpyAsync(perm, plan->perm, R * 4, cudaMemcpyDeviceToDevice, s), "copy perm");
+  return MOE_OK;
+}
+
+moe_status moe_status_sync(moe_plan_t *plan, moe_stream_t stream) {
+  g_last_error.clear();
+  if (!plan) return fail(MOE_ERR_INVALID_ARG, "plan is NULL");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  MOE_CUDA(cudaStreamSynchronize(s), "stream synchronize");
+  DevStatus h;
+  MOE_CUDA(cudaMemcpy(&h, plan->status, sizeof h, cudaMemcpyDeviceToHost), "read status");
+  if (h.code == kDevOk) return MOE_OK;
+  // clear the status and the grid barrier so the plan can be used again
+  MOE_CUDA(cudaMemset(plan->status, 0, sizeof(DevStatus)), "clear status");
+  MOE_CUDA(cudaMemset(plan->barrier, 0, 16), "clear barrier");
+  MOE_CUDA(cudaDeviceSynchronize(), "synchronize");
+  if (h.code == kDevTimeout)
+    return fail(MOE_ERR_DEVICE_TIMEOUT, "device wait ran out (site %u, block %u)", h.where, h.detail);
+  return fail(MOE_ERR_DEVICE_BOUNDS, "device index out of range (site %u, value %u)", h.where, h.detail);
+}
+
+}  // extern "C"

@@ -1,0 +1,60 @@
+// combine.cu -- deterministic combine of the expert outputs of each token.
+//
+// out_t = bf16( [x_t +] 2^{2e_t} * ( sum_{j=0}^{k-1} Y[inv[t*k+j]] + Y[R+t] ) )
+// The routed rows of Y already carry their routing weight; the shared expert's
+// row (the expert that sees every token, "Perplexity open sources Lily...",
+// section "Requirements and model layout") enters with weight 1. The sum runs in
+// this fixed order in fp32 with one final rounding, so the result does not
+// depend on scheduling (no floating-point atomics).
+#include "kernels.cuh"
+
+namespace moe {
+
+__global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
+  const int t = blockIdx.x;
+  const int H = a.H, k = a.k;
+  __shared__ int rows[kMaxTopK + 1];
+  if (threadIdx.x < k) rows[threadIdx.x] = a.inv[static_cast<size_t>(t) * k + threadIdx.x];
+  if (threadIdx.x == 0) rows[k] = a.R + t;
+  __syncthreads();
+  const int e2 = 2 * a.xexp[t];
+  for (int c = threadIdx.x; c < H / 8; c += blockDim.x) {
+    float acc[8];
+#pragma unroll
+    for (int q = 0; q < 8; ++q) acc[q] = 0.f;
+    for (int j = 0; j <= k; ++j) {
+      const uint4 v = __ldcs(reinterpret_cast<const uint4 *>(a.y + static_cast<size_t>(rows[j]) * H) + c);
+      const __half2 *hv = reinterpret_cast<const __half2 *>(&v);
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float2 f = __half22float2(hv[q]);
+        acc[2 * q] += f.x;
+        acc[2 * q + 1] += f.y;
+      }
+    }
+    uint4 res;
+    uint32_t *rp = reinterpret_cast<uint32_t *>(&res);
+    uint4 xr = make_uint4(0, 0, 0, 0);
+    if (a.residual) xr = *(reinterpret_cast<const uint4 *>(a.residual + static_cast<size_t>(t) * H) + c);
+    const uint32_t *xp = reinterpret_cast<const uint32_t *>(&xr);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      float lo = ldexpf(acc[2 * q], e2), hi = ldexpf(acc[2 * q + 1], e2);
+      if (a.residual) {
+        lo += __uint_as_float(xp[q] << 16);
+        hi += __uint_as_float(xp[q] & 0xffff0000u);
+      }
+      rp[q] = static_cast<uint32_t>(float_to_bf16_bits(lo)) |
+              (static_cast<uint32_t>(float_to_bf16_bits(hi)) << 16);
+    }
+    *(reinterpret_cast<uint4 *>(a.out + static_cast<size_t>(t) * H) + c) = res;
+  }
+}
+
+cudaError_t launch_combine(const CombineArgs &a, cudaStream_t s) {
+  if (a.T <= 0) return cudaSuccess;
+  combine_kernel<<<a.T, 256, 0, s>>>(a);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

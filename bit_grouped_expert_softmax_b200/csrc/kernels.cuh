@@ -1,0 +1,97 @@
+// kernels.cuh -- argument blocks and launch declarations of the MoE kernels.
+#pragma once
+
+#include "common.cuh"
+
+namespace moe {
+
+constexpr int kTileM = 128;  // weight rows per grouped-GEMM tile (MMA M)
+constexpr int kTileN = 128;  // activation rows per grouped-GEMM tile (MMA N, max)
+constexpr int kTileK = 64;   // K elements per pipeline stage (one 128-byte fp16 row)
+
+struct RouteScanArgs {
+  int T, E, k, H, I, Is, nchunk;
+  int32_t *chunk_cnt;   // [nchunk][E] counts in, bases out
+  int32_t *offsets;     // [E+1]
+  WorkItem *gu_items;   // gate/up work list
+  int max_gu;
+  WorkItem *dn_items;   // down work list
+  int max_dn;
+  int32_t *item_counts; // [0] gate/up items, [1] down items
+  DevStatus *status;
+};
+
+struct RouteScatterArgs {
+  int T, E, k, H;
+  const int32_t *ids;         // [T*k]
+  const int32_t *chunk_base;  // [nchunk][E]
+  int32_t *perm;              // [T*k]
+  int32_t *inv;               // [T*k]
+  const uint16_t *x;          // [T, H] bf16, or null (routing only)
+  __half *xt;                 // [T*k + T, H] gathered fp16 rows
+  int32_t *xexp;              // [T] power-of-two exponent of each token's row scale
+  DevStatus *status;
+};
+
+// Weights of one layer (device pointers, layout of the public header).
+struct LayerWeights {
+  const uint32_t *packed;
+  const uint16_t *scales;
+  const uint16_t *biases;
+  const uint32_t *sh_packed;
+  const uint16_t *sh_scales;
+  const uint16_t *sh_biases;
+};
+
+struct GemmArgs {
+  int T, E, k, H, I, Is;
+  int R;                    // T*k routed rows; shared rows follow at R..R+T-1
+  LayerWeights w;
+  const __half *xt;         // [R+T, H] gathered activations (gate/up operand)
+  __half *h;                // routed rows [R, I] at h, shared rows [T, Is] at h + h_shared_off
+  int64_t h_shared_off;     // elements
+  __half *y;                // [R+T, H] weighted expert outputs (down result)
+  const int32_t *perm;      // [R] row -> flat index t*k+j
+  const float *wts;         // [T*k] routing weights by flat index
+  const int32_t *xexp;      // [T]
+  const WorkItem *items;
+  const int32_t *item_count;
+  int max_items;
+  DevStatus *status;
+};
+
+struct CombineArgs {
+  int T, k, H, R;
+  const int32_t *inv;        // [T*k] flat index -> row
+  const __half *y;           // [R+T, H]
+  const int32_t *xexp;       // [T]
+  const uint16_t *residual;  // [T, H] bf16 or null
+  uint16_t *out;             // [T, H] bf16 (may alias residual)
+};
+
+struct SmallTArgs {
+  int T, E, k, H, I, Is;
+  const uint16_t *x;        // [T, H] bf16
+  const float *logits;      // [T, E]
+  LayerWeights w;
+  float *hbuf;              // [(T*k+1), T, max(I,Is)] fp32 scratch
+  uint32_t *barrier;        // grid barrier {count, generation}
+  const uint16_t *residual; // [T, H] or null
+  uint16_t *out;            // [T, H]
+  DevStatus *status;
+};
+
+__global__ void route_topk_kernel(int T, int E, int k, const float *__restrict__ logits,
+                                  int32_t *__restrict__ ids, float *__restrict__ wts,
+                                  int32_t *__restrict__ chunk_cnt);
+__global__ void route_scan_kernel(RouteScanArgs a);
+__global__ void route_scatter_kernel(RouteScatterArgs a);
+
+// host-side launchers (each returns the launch's cudaError_t)
+cudaError_t launch_gemm_gate_up(const GemmArgs &a, int num_sms, cudaStream_t s);
+cudaError_t launch_gemm_down(const GemmArgs &a, int num_sms, cudaStream_t s);
+cudaError_t launch_combine(const CombineArgs &a, cudaStream_t s);
+cudaError_t launch_small_t(const SmallTArgs &a, int num_sms, cudaStream_t s);
+int small_t_grid(int num_sms);
+
+}  // namespace moe

@@ -1,0 +1,227 @@
+// route.cu -- routing on the device, one stream, no host synchronisation.
+//
+// The report lists the routing histogram, prefix scan, scatter and block map
+// as work kept inside one GPU command buffer (aioga.com record, article body
+// paragraph 5); the router itself scores every expert and keeps the top k
+// ("Perplexity open sources Lily...", section "Requirements and model layout").
+// Three kernels:
+//   route_topk_kernel    softmax over E, warp top-k, renormalised weights,
+//                        per-chunk expert histogram
+//   route_scan_kernel    per-expert totals, exclusive scan (offsets), per-chunk
+//                        bases, and the grouped-GEMM work lists (block map)
+//   route_scatter_kernel stable permutation (experts ascending, tokens ascending
+//                        within an expert), its inverse, and the gather of the
+//                        activations into expert-contiguous fp16 rows
+#include "kernels.cuh"
+#include "topk.cuh"
+
+namespace moe {
+
+__global__ void __launch_bounds__(256) route_topk_kernel(int T, int E, int k,
+                                                         const float *__restrict__ logits,
+                                                         int32_t *__restrict__ ids,
+                                                         float *__restrict__ wts,
+                                                         int32_t *__restrict__ chunk_cnt) {
+  __shared__ int cnt[kMaxExperts];
+  const int chunk = blockIdx.x;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
+  __syncthreads();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t0 = chunk * kRouteChunk;
+  const int t1 = min(T, t0 + kRouteChunk);
+  for (int t = t0 + warp; t < t1; t += blockDim.x / 32) {
+    int id;
+    float w;
+    warp_topk(logits + static_cast<size_t>(t) * E, E, k, lane, id, w);
+    if (lane < k) {
+      ids[static_cast<size_t>(t) * k + lane] = id;
+      wts[static_cast<size_t>(t) * k + lane] = w;
+      atomicAdd(&cnt[id], 1);  // integer counts: order-independent
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) chunk_cnt[static_cast<size_t>(chunk) * E + e] = cnt[e];
+}
+
+// Single block. Turns per-chunk counts into per-chunk bases (in place), writes
+// offsets[0..E] and the two work lists.
+__global__ void __launch_bounds__(1024) route_scan_kernel(RouteScanArgs a) {
+  __shared__ int tot[kMaxExperts + 1];
+  __shared__ int off[kMaxExperts + 2];
+  __shared__ int gu_off[kMaxExperts + 2];
+  __shared__ int dn_off[kMaxExperts + 2];
+  __shared__ int warp_tot[3][32];
+  const int E = a.E;
+  const int G = E + 1;  // routed experts plus the shared one
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int run = 0;
+    for (int c = 0; c < a.nchunk; ++c) {
+      int32_t *p = a.chunk_cnt + static_cast<size_t>(c) * E + e;
+      const int v = *p;
+      *p = run;
+      run += v;
+    }
+    tot[e] = run;
+  }
+  __syncthreads();
+  // exclusive scans over the groups, done by warp 0 with 9 values per lane (G <= 257)
+  if (threadIdx.x < 32) {
+    const int lane = threadIdx.x;
+    constexpr int PER = (kMaxExperts + 1 + 31) / 32;
+    int cnt[PER], gu[PER], dn[PER];
+    int sc = 0, sg = 0, sd = 0;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      const int g = lane * PER + i;
+      int n = 0, gi = 0, di = 0;
+      if (g < G) {
+        n = (g < E) ? tot[g] : a.T;
+        const int ntile = (n + kTileN - 1) / kTileN;
+        gi = ntile * ((g < E ? a.I : a.Is) / kTileM);
+        di = ntile * (a.H / kTileM);
+      }
+      cnt[i] = (g < E) ? n : 0;
+      gu[i] = gi;
+      dn[i] = di;
+      sc += cnt[i];
+      sg += gi;
+      sd += di;
+    }
+    const int ic = warp_incl_scan(sc), ig = warp_incl_scan(sg), id = warp_incl_scan(sd);
+    int bc = ic - sc, bg = ig - sg, bd = id - sd;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      const int g = lane * PER + i;
+      if (g <= G) {
+        off[g] = bc;
+        gu_off[g] = bg;
+        dn_off[g] = bd;
+      }
+      bc += cnt[i];
+      bg += gu[i];
+      bd += dn[i];
+    }
+    if (lane == 31) {
+      warp_tot[0][0] = ic;
+      warp_tot[1][0] = ig;
+      warp_tot[2][0] = id;
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e <= E; e += blockDim.x) a.offsets[e] = (e < E) ? off[e] : a.T * a.k;
+  // per-chunk bases become absolute row positions
+  for (int i = threadIdx.x; i < a.nchunk * E; i += blockDim.x) a.chunk_cnt[i] += off[i % E];
+  // work lists: group g's tiles are (n-tile, m-block) with the m-block fastest,
+  // so neighbouring CTAs share the activation tile of one n-tile
+  const int R = a.T * a.k;
+  const int gu_total = warp_tot[1][0], dn_total = warp_tot[2][0];
+  if (threadIdx.x == 0) {
+    if (gu_total > a.max_gu || dn_total > a.max_dn)
+      report_error(a.status, kDevBounds, 10, static_cast<uint32_t>(max(gu_total, dn_total)));
+    a.item_counts[0] = min(gu_total, a.max_gu);
+    a.item_counts[1] = min(dn_total, a.max_dn);
+  }
+  for (int g = threadIdx.x >> 5; g < G; g += blockDim.x >> 5) {
+    const int lane = threadIdx.x & 31;
+    const int n = (g < E) ? tot[g] : a.T;
+    const int row0 = (g < E) ? off[g] : R;
+    const int ntile = (n + kTileN - 1) / kTileN;
+    const int mg = (g < E ? a.I : a.Is) / kTileM, md = a.H / kTileM;
+    for (int i = lane; i < ntile * mg; i += 32) {
+      const int nt = i / mg, mb = i % mg, slot = gu_off[g] + i;
+      if (slot < a.max_gu)
+        a.gu_items[slot] = WorkItem{g, row0 + nt * kTileN, min(kTileN, n - nt * kTileN), mb};
+    }
+    for (int i = lane; i < ntile * md; i += 32) {
+      const int nt = i / md, mb = i % md, slot = dn_off[g] + i;
+      if (slot < a.max_dn)
+        a.dn_items[slot] = WorkItem{g, row0 + nt * kTileN, min(kTileN, n - nt * kTileN), mb};
+    }
+  }
+}
+
+// Stable scatter plus gather. One block per routing chunk of 32 tokens.
+__global__ void __launch_bounds__(256) route_scatter_kernel(RouteScatterArgs a) {
+  __shared__ int cnt[kMaxExperts];
+  __shared__ int pos_s[kRouteChunk * kMaxTopK];
+  const int chunk = blockIdx.x, E = a.E, k = a.k, T = a.T;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = a.chunk_base[static_cast<size_t>(chunk) * E + e];
+  __syncthreads();
+  const int t0 = chunk * kRouteChunk, t1 = min(T, t0 + kRouteChunk);
+  const int f0 = t0 * k, f1 = t1 * k;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (warp == 0) {
+    // flat order f = t*k + j is token-ascending; within a batch of 32 entries the
+    // rank among equal experts comes from match/popc, across batches from cnt[]
+    for (int fb = f0; fb < f1; fb += 32) {
+      const int f = fb + lane;
+      const bool valid = f < f1;
+      const unsigned active = __ballot_sync(0xffffffffu, valid);
+      if (valid) {
+        const int e = a.ids[f];
+        const unsigned peers = __match_any_sync(active, e);
+        const int rank = __popc(peers & ((1u << lane) - 1u));
+        const int base = cnt[e];
+        __syncwarp(active);
+        if (rank == 0) cnt[e] = base + __popc(peers);
+        const int pos = base + rank;
+        if (pos < 0 || pos >= T * k) {
+          report_error(a.status, kDevBounds, 20, static_cast<uint32_t>(pos));
+        } else {
+          a.perm[pos] = f;
+          a.inv[f] = pos;
+        }
+        pos_s[f - f0] = pos;
+      }
+      __syncwarp();
+    }
+  }
+  if (a.x == nullptr) return;
+  __syncthreads();
+  // gather: one warp per token; the row is scaled by a power of two 2^-e chosen
+  // from its max |x| (exact in fp16 unless the row spans more than fp16's range),
+  // converted to fp16 and written, in the K-permuted operand order, to the
+  // token's k routed rows and its shared-expert row
+  const int H = a.H, R = T * k;
+  const int nchunk8 = H / 8;
+  for (int t = t0 + warp; t < t1; t += blockDim.x / 32) {
+    const uint4 *src = reinterpret_cast<const uint4 *>(a.x + static_cast<size_t>(t) * H);
+    float amax = 0.f;
+    for (int c = lane; c < nchunk8; c += 32) {
+      const uint4 v = __ldg(src + c);
+      const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        amax = fmaxf(amax, fabsf(__uint_as_float(w4[q] << 16)));
+        amax = fmaxf(amax, fabsf(__uint_as_float(w4[q] & 0xffff0000u)));
+      }
+    }
+    amax = warp_max(amax);
+    int ex = 0;
+    if (amax > 0.f && amax <= 3.0e38f) ex = min(max(ilogbf(amax) - 1, -100), 100);  // scaled max in [2, 4)
+    const float scale = exp2f(static_cast<float>(-ex));
+    if (lane == 0) a.xexp[t] = ex;
+    for (int c = lane; c < nchunk8; c += 32) {
+      const uint4 v = __ldg(src + c);
+      const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+      __half hv[8];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        hv[2 * q] = __float2half_rn(__uint_as_float(w4[q] << 16) * scale);
+        hv[2 * q + 1] = __float2half_rn(__uint_as_float(w4[q] & 0xffff0000u) * scale);
+      }
+      uint4 o;
+      uint32_t *op = reinterpret_cast<uint32_t *>(&o);
+#pragma unroll
+      for (int s = 0; s < 8; s += 2) op[s / 2] = pack_half2(hv[kperm_src(s)], hv[kperm_src(s + 1)]);
+      for (int j = 0; j < k; ++j) {
+        const int row = pos_s[(t - t0) * k + j];
+        if (row >= 0 && row < R)
+          reinterpret_cast<uint4 *>(a.xt + static_cast<size_t>(row) * H)[c] = o;
+      }
+      reinterpret_cast<uint4 *>(a.xt + static_cast<size_t>(R + t) * H)[c] = o;
+    }
+  }
+}
+
+}  // namespace moe

@@ -1,0 +1,185 @@
+"""CUDA path against the fp64 oracle, through the C ABI (needs a B200)."""
+
+import numpy as np
+import pytest
+
+import oracle
+from bit_grouped_expert_softmax_b200 import api, synth
+from helpers import check_output, to_device
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+
+def _layer(inp):
+    return api.DeviceLayer.from_inputs(inp)
+
+
+def _plan(inp, T_max=None, flags=0):
+    return api.Plan(T_max or max(1, inp.T), inp.H, inp.E, inp.k, inp.I, inp.Is, flags)
+
+
+def _forward(plan, inp, layer=None):
+    layer = layer or _layer(inp)
+    x, logits = to_device(inp)
+    out = plan.forward(x, logits, layer)
+    plan.status_sync()
+    return out.cpu().numpy()
+
+
+_INPUT_CACHE = {}
+
+
+def workload(name):
+    if name not in _INPUT_CACHE:
+        _INPUT_CACHE[name] = synth.make_workload(name)
+    return _INPUT_CACHE[name]
+
+
+def stack_logits(layer, T=None):
+    w = synth.WORKLOADS["stack"]
+    rng = np.random.default_rng([w.seed, layer])
+    return synth.draw_logits(rng, w.T if T is None else T, w.E, w.k, w.logit_std, w.zipf_s)
+
+
+# ----------------------------------------------------------------------------
+# routing: ids, offsets and permutation bit-exact; weights to fp32 rounding
+# ----------------------------------------------------------------------------
+
+def _check_route(logits, k, plan):
+    ids, w, offsets, perm = plan.route(torch.from_numpy(logits).cuda())
+    plan.status_sync()
+    r_ids, r_w, _, r_off, r_perm = oracle.route(logits, k)
+    assert np.array_equal(ids.cpu().numpy(), r_ids)
+    assert np.array_equal(offsets.cpu().numpy(), r_off)
+    assert np.array_equal(perm.cpu().numpy(), r_perm)
+    np.testing.assert_allclose(w.cpu().numpy(), r_w, rtol=2e-6, atol=1e-7)
+
+
+@pytest.mark.parametrize("name", ["tiny", "decode", "prefill", "zipf"])
+def test_route_bit_exact(name):
+    wl = synth.WORKLOADS[name]
+    rng = np.random.default_rng(wl.seed)
+    _ = rng.standard_normal((wl.T, wl.H), dtype=np.float32)  # x is drawn first
+    logits = synth.draw_logits(rng, wl.T, wl.E, wl.k, wl.logit_std, wl.zipf_s)
+    assert np.array_equal(logits, workload(name).logits) if name in ("tiny", "decode") else True
+    plan = api.Plan(wl.T, wl.H, wl.E, wl.k, wl.I, wl.Is)
+    _check_route(logits, wl.k, plan)
+
+
+@pytest.mark.parametrize("layer", [0, 39])
+def test_route_bit_exact_stack_chunk(layer):
+    wl = synth.WORKLOADS["stack"]
+    plan = api.Plan(wl.T, wl.H, wl.E, wl.k, wl.I, wl.Is)
+    _check_route(stack_logits(layer), wl.k, plan)
+
+
+def test_route_ties_and_extremes():
+    E, k, T = 64, 8, 40
+    rng = np.random.default_rng(5)
+    logits = rng.standard_normal((T, E)).astype(np.float32)
+    logits[0] = 1.0                       # all equal: ids 0..7
+    logits[1, ::2] = 3.0                  # ties among the top
+    logits[2] = -1e30                     # huge negative values
+    logits[2, 5] = 0.0
+    logits[3, 10] = 1e30                  # one dominant expert
+    plan = api.Plan(T, 256, E, k, 128, 128)
+    _check_route(logits, k, plan)
+
+
+# ----------------------------------------------------------------------------
+# whole layer
+# ----------------------------------------------------------------------------
+
+def test_forward_tiny():
+    inp = workload("tiny")
+    check_output(_forward(_plan(inp), inp), oracle.moe_forward(inp), "tiny")
+
+
+def test_forward_decode():
+    inp = workload("decode")
+    check_output(_forward(_plan(inp), inp), oracle.moe_forward(inp), "decode")
+
+
+def test_forward_mid_size_ragged():
+    """Several n-tiles per expert with ragged tails, several m-blocks, Is != I."""
+    inp = synth.make_layer(300, 512, 32, 4, 256, 384, seed=21, logit_std=1.0)
+    check_output(_forward(_plan(inp), inp), oracle.moe_forward(inp), "mid")
+
+
+@pytest.mark.parametrize("name,nrows", [("prefill", 96), ("zipf", 96)])
+def test_forward_full_size_sampled_rows(name, nrows):
+    inp = workload(name)
+    got = _forward(_plan(inp), inp)
+    rng = np.random.default_rng(99)
+    rows = np.unique(np.concatenate([[0, inp.T - 1], rng.choice(inp.T, nrows - 2, replace=False)]))
+    ref = oracle.moe_forward(inp, x=inp.x[rows], logits=inp.logits[rows])
+    check_output(got[rows], ref, name)
+
+
+@pytest.mark.parametrize("T", [1, 2, 3, 5, 8, 9])
+@pytest.mark.parametrize("flags", [0, api.MOE_FLAG_FORCE_GROUPED])
+def test_forward_small_batches(T, flags):
+    inp = synth.make_layer(T, 2048, 256, 8, 512, 512, seed=100 + T, logit_std=2.0)
+    check_output(_forward(_plan(inp, flags=flags), inp), oracle.moe_forward(inp), f"T={T} flags={flags}")
+
+
+def test_one_expert_takes_every_token():
+    inp = synth.make_layer(150, 256, 16, 2, 128, 128, seed=31)
+    inp.logits[:, 3] += 100.0  # expert 3 is everyone's first choice; most experts get nothing
+    check_output(_forward(_plan(inp), inp), oracle.moe_forward(inp), "hot expert")
+
+
+def test_deterministic_reruns():
+    inp = workload("prefill")
+    plan = _plan(inp)
+    layer = _layer(inp)
+    a = _forward(plan, inp, layer)
+    b = _forward(plan, inp, layer)
+    assert np.array_equal(a, b)
+
+
+def test_forward_host_matches_device_call():
+    inp = workload("tiny")
+    plan = _plan(inp)
+    layer = _layer(inp)
+    dev = _forward(plan, inp, layer)
+    x = torch.from_numpy(inp.x.view(np.int16)).pin_memory()
+    lg = torch.from_numpy(inp.logits).pin_memory()
+    out = torch.empty_like(x).pin_memory()
+    api.moe_forward_host(plan.handle, inp.T, x, lg, *layer.args(), out)
+    assert np.array_equal(out.numpy(), dev)
+
+
+def test_output_canaries_untouched():
+    inp = workload("tiny")
+    plan = _plan(inp)
+    x, logits = to_device(inp)
+    guard = 4096
+    buf = torch.full((inp.T * inp.H + 2 * guard,), 0x5A5A, dtype=torch.int16, device="cuda")
+    out = buf[guard:guard + inp.T * inp.H].view(inp.T, inp.H)
+    api.moe_forward(plan.handle, inp.T, x, logits, *_layer(inp).args(), out)
+    plan.status_sync()
+    b = buf.cpu().numpy()
+    assert np.all(b[:guard] == 0x5A5A) and np.all(b[-guard:] == 0x5A5A)
+
+
+def test_empty_batch_is_a_no_op():
+    inp = workload("tiny")
+    plan = _plan(inp)
+    x, logits = to_device(inp)
+    api.moe_forward(plan.handle, 0, x, logits, *_layer(inp).args(), torch.empty_like(x))
+    plan.status_sync()
+
+
+def test_invalid_arguments_enqueue_nothing():
+    inp = workload("tiny")
+    plan = _plan(inp)
+    x, logits = to_device(inp)
+    with pytest.raises(api.MoEError) as ei:
+        api.moe_forward(plan.handle, inp.T + 1, x, logits, *_layer(inp).args(), torch.empty_like(x))
+    assert ei.value.status == -1
+    with pytest.raises(api.MoEError):
+        api.moe_forward(plan.handle, inp.T, x, logits, *_layer(inp).args(), x)  # out aliases x
+    plan.status_sync()
