@@ -154,7 +154,8 @@ def run_gpu(args, rank, world, local_rank):
         logits = torch.from_numpy(inp.logits).to(dev)
         out = torch.empty_like(x)
         plan = api.Plan(inp.T, inp.H, inp.E, inp.k, inp.I, inp.Is)
-        stream = torch.cuda.current_stream(dev)
+        stream = torch.cuda.Stream(dev)  # graphs cannot be captured on the default stream
+        torch.cuda.set_stream(stream)
         launches_per_step = 1 if inp.T <= 8 else 6
 
         def step(i):

@@ -177,6 +177,9 @@ moe_status enqueue_layer(moe_plan_s *p, int T, const uint16_t *x, const float *l
   g.w = w; g.xt = p->xt; g.h = p->h;
   g.h_shared_off = static_cast<int64_t>(p->T_max) * p->k * p->I;
   g.y = p->y; g.perm = p->perm; g.wts = p->wts; g.xexp = p->xexp; g.status = p->status;
+  g.xt_rows = static_cast<int64_t>(p->T_max) * (p->k + 1);
+  g.h_rows = static_cast<int64_t>(p->T_max) * p->k;
+  g.hs_rows = p->T_max;
   g.items = p->gu_items;
   g.item_count = p->item_counts;
   g.max_items = static_cast<int>(max_gu_items(T, p->E, p->k, p->I, p->Is));

@@ -57,6 +57,9 @@ struct GemmArgs {
   const WorkItem *items;
   const int32_t *item_count;
   int max_items;
+  int64_t xt_rows;          // rows allocated for xt (tensor-map extent)
+  int64_t h_rows;           // routed h rows allocated
+  int64_t hs_rows;          // shared h rows allocated
   DevStatus *status;
 };
 
