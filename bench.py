@@ -156,7 +156,7 @@ def run_gpu(args, rank, world, local_rank):
         plan = api.Plan(inp.T, inp.H, inp.E, inp.k, inp.I, inp.Is)
         stream = torch.cuda.Stream(dev)  # graphs cannot be captured on the default stream
         torch.cuda.set_stream(stream)
-        launches_per_step = 1 if inp.T <= 8 else 6
+        launches_per_step = 1 if inp.T <= 8 else 7
 
         def step(i):
             api.moe_forward(plan.handle, inp.T, x, logits, *reps[i % n_rep].args(), out, stream)
@@ -216,6 +216,15 @@ def run_gpu(args, rank, world, local_rank):
             api.moe_forward_host(plan.handle, inp.T, xh, lh, *reps[i % n_rep].args(), oh, stream)
         e2e_s = (time.perf_counter() - t0) / n_e2e
         plan.status_sync(stream)
+        # per-kernel times: the same steps launched eagerly with the library's
+        # CUDA events around every kernel, on the launching stream
+        api.moe_profile_enable(plan.handle, 8 * max(steps, n_rep))
+        torch.cuda.synchronize(dev)
+        for i in range(max(steps, n_rep)):
+            step(i)
+        prof = api.moe_profile_read(plan.handle, stream)
+        api.moe_profile_enable(plan.handle, 0)
+        plan.status_sync(stream)
         achieved_gbs = rf["weight_bytes"] / (ms_step * 1e-3) / 1e9
         achieved_tf = rf["flops"] / (ms_step * 1e-3) / 1e12
         res = dict(workload=name, T=inp.T, ms_per_step=ms_step, tokens_s=tokens_s, rf=rf,
@@ -223,7 +232,7 @@ def run_gpu(args, rank, world, local_rank):
                    graph=graph is not None, timed_steps=timed_steps, clocks=clk.summary(),
                    e2e_tokens_s=inp.T * world / e2e_s,
                    h2d=inp.T * inp.H * 2 + inp.T * inp.E * 4, d2h=inp.T * inp.H * 2,
-                   launches=launches_per_step * timed_steps, inp=inp)
+                   launches=launches_per_step * timed_steps, inp=inp, prof=prof)
         del graph
         plan.close()
         return res
@@ -238,23 +247,43 @@ def run_gpu(args, rank, world, local_rank):
     return main, extra, peaks, peaks_kind
 
 
+KERNEL_SHARE = {"small_t": (1.0, 1.0), "gate_up": (2 / 3, 2 / 3), "down": (1 / 3, 1 / 3)}
+
+
+def kernel_table(r):
+    prof = r["prof"]
+    tot = sum(v[0] for v in prof.values()) or 1.0
+    return {k: {"launches": n, "avg_us": round(1e3 * ms / max(n, 1), 3), "share": round(ms / tot, 4)}
+            for k, (ms, n) in sorted(prof.items(), key=lambda kv: -kv[1][0])}
+
+
 def roofline_obj(r, peaks, peaks_kind):
+    """Roofline of the dominant kernel: its algorithmic bytes or FLOPs per launch
+    over its average launch time (library CUDA events on the launch stream)."""
     rf = r["rf"]
-    if rf["bound"] == "hbm":
-        a, p, unit = r["achieved_gbs"], peaks["hbm_gbs"], "GB/s"
+    prof = r["prof"]
+    name = max(prof, key=lambda k: prof[k][0])
+    ms, n = prof[name]
+    avg_s = ms * 1e-3 / max(n, 1)
+    fb, ff = KERNEL_SHARE.get(name, (0.0, 0.0))
+    kbytes, kflops = rf["weight_bytes"] * fb, rf["flops"] * ff
+    t_hbm = kbytes / (peaks["hbm_gbs"] * 1e9)
+    t_tc = kflops / (peaks["bf16_tflops"] * 1e12)
+    if t_hbm >= t_tc:
+        a, p, unit, bound = kbytes / avg_s / 1e9, peaks["hbm_gbs"], "GB/s", "hbm"
     else:
-        a, p, unit = r["achieved_tflops"], peaks["bf16_tflops"], "TFLOP/s"
-    return {"bound": rf["bound"], "achieved": round(a, 2), "peak": p, "unit": unit, "frac": round(a / p, 4),
-            "traffic": None, "peak_source": peaks_kind,
-            "algorithmic": {"weight_bytes": rf["weight_bytes"], "flops": rf["flops"],
-                            "touched_experts_incl_shared": rf["touched"]},
-            "kernel": "whole layer step (all kernels)"}
+        a, p, unit, bound = kflops / avg_s / 1e12, peaks["bf16_tflops"], "TFLOP/s", "tensor"
+    return {"bound": bound, "achieved": round(a, 2), "peak": p, "unit": unit, "frac": round(a / p, 4),
+            "traffic": None, "peak_source": peaks_kind, "kernel": name, "kernel_avg_us": round(avg_s * 1e6, 3),
+            "algorithmic_per_launch": {"weight_bytes": int(kbytes), "flops": kflops,
+                                       "touched_experts_incl_shared": rf["touched"]}}
 
 
 def summarize_extra(r, peaks, peaks_kind):
     return {"T": r["T"], "tokens_s": round(r["tokens_s"], 1), "ms_per_step": round(r["ms_per_step"], 5),
             "effective_tflops": round(r["achieved_tflops"], 2), "achieved_weight_gbs": round(r["achieved_gbs"], 1),
-            "roofline": roofline_obj(r, peaks, peaks_kind), "graph": r["graph"], "clocks": r["clocks"],
+            "roofline": roofline_obj(r, peaks, peaks_kind), "kernels": kernel_table(r), "graph": r["graph"],
+            "clocks": r["clocks"],
             "e2e_tokens_s": round(r["e2e_tokens_s"], 1)}
 
 
@@ -347,6 +376,7 @@ def main():
                     f"({r['n_rep']} x {r['rf']['weight_bytes'] / 1e6:.1f} MB touched > 4 x L2)"),
                     graph=r["graph"]),
                 "roofline": roofline_obj(r, peaks, peaks_kind),
+                "kernels": kernel_table(r),
                 "effective_tflops": round(r["achieved_tflops"], 3),
                 "cpu_baseline": cpu,
                 "e2e": {"value": round(r["e2e_tokens_s"], 1), "unit": "tokens/s",

@@ -58,10 +58,12 @@ def load():
     lib.moe_stack_forward.argtypes = [P, I, I, P, P, ctypes.POINTER(moe_layer_weights), P]
     lib.moe_route.argtypes = [P, I, P, P, P, P, P, P]
     lib.moe_status_sync.argtypes = [P, P]
+    lib.moe_profile_enable.argtypes = [P, I]
+    lib.moe_profile_read.argtypes = [P, P, P, P]
     lib.moe_last_error.restype = ctypes.c_char_p
     lib.moe_version.restype = ctypes.c_char_p
     for name in ("moe_plan", "moe_plan_destroy", "moe_forward", "moe_forward_host", "moe_stack_forward",
-                 "moe_route", "moe_status_sync"):
+                 "moe_route", "moe_status_sync", "moe_profile_enable", "moe_profile_read"):
         getattr(lib, name).restype = I
     _lib = lib
     return lib
@@ -144,6 +146,21 @@ def moe_route(plan, T, logits, ids=None, w=None, offsets=None, perm=None, stream
 
 def moe_status_sync(plan, stream=None):
     _check(load().moe_status_sync(plan, _stream(stream)))
+
+
+KERNEL_NAMES = ["route_topk", "route_scan", "route_scatter", "gather", "gate_up", "down", "combine", "small_t"]
+
+
+def moe_profile_enable(plan, max_launches):
+    _check(load().moe_profile_enable(plan, max_launches))
+
+
+def moe_profile_read(plan, stream=None):
+    """{kernel name: (total ms, launches)} since the last read."""
+    ms = (ctypes.c_double * len(KERNEL_NAMES))()
+    n = (ctypes.c_int32 * len(KERNEL_NAMES))()
+    _check(load().moe_profile_read(plan, _stream(stream), ms, n))
+    return {name: (ms[i], n[i]) for i, name in enumerate(KERNEL_NAMES) if n[i]}
 
 
 # ----------------------------------------------------------------------------

@@ -7,12 +7,14 @@
 #include <cstdio>
 #include <cstring>
 #include <string>
+#include <vector>
 
 #include "../../include/moe_b200.h"
 #include "kernels.cuh"
 
 namespace moe {
 size_t small_t_smem_bytes(int T, int H, int k, int I, int Is);
+void set_last_error(const char *msg);
 }
 
 using namespace moe;
@@ -20,6 +22,12 @@ using namespace moe;
 namespace {
 
 thread_local std::string g_last_error;
+
+}  // namespace
+
+void moe::set_last_error(const char *msg) { g_last_error = msg; }
+
+namespace {
 
 moe_status fail(moe_status st, const char *fmt, ...) {
   char buf[512];
@@ -86,6 +94,10 @@ struct moe_plan_s {
   float *logits_stage;
   uint16_t *out_stage;
   int64_t max_gu, max_dn;
+  // per-kernel timing (moe_profile_enable / moe_profile_read)
+  std::vector<cudaEvent_t> prof_events;  // 2 per recorded launch
+  std::vector<int> prof_kind;
+  int prof_used = 0;
 };
 
 namespace {
@@ -135,25 +147,57 @@ LayerWeights make_weights(const void *packed, const void *scales, const void *bi
   return w;
 }
 
-// routing kernels: ids/weights, histogram + scan + work lists, scatter (+ gather if x)
+// Brackets one kernel launch with the plan's profiling events, if enabled.
+struct ProfScope {
+  moe_plan_s *p;
+  cudaStream_t s;
+  int slot = -1;
+  ProfScope(moe_plan_s *p_, int kind, cudaStream_t s_) : p(p_), s(s_) {
+    if (p->prof_used < static_cast<int>(p->prof_kind.size())) {
+      slot = p->prof_used++;
+      p->prof_kind[slot] = kind;
+      cudaEventRecord(p->prof_events[2 * slot], s);
+    }
+  }
+  ~ProfScope() {
+    if (slot >= 0) cudaEventRecord(p->prof_events[2 * slot + 1], s);
+  }
+};
+
+// routing kernels: ids/weights + histogram, scan + work lists, scatter, gather (if x)
 moe_status enqueue_routing(moe_plan_s *p, int T, const float *logits, const uint16_t *x, cudaStream_t s) {
   const int nchunk = static_cast<int>(cdiv(T, kRouteChunk));
-  route_topk_kernel<<<nchunk, 256, 0, s>>>(T, p->E, p->k, logits, p->ids, p->wts, p->chunk);
-  MOE_CUDA(cudaGetLastError(), "route_topk launch");
+  const int tok_blocks = static_cast<int>(cdiv(T, 8));
+  {
+    ProfScope ps(p, MOE_KERNEL_ROUTE_TOPK, s);
+    route_topk_kernel<<<tok_blocks, 256, 0, s>>>(T, p->E, p->k, logits, p->ids, p->wts, p->chunk);
+    MOE_CUDA(cudaGetLastError(), "route_topk launch");
+  }
   RouteScanArgs sa;
   sa.T = T; sa.E = p->E; sa.k = p->k; sa.H = p->H; sa.I = p->I; sa.Is = p->Is; sa.nchunk = nchunk;
   sa.chunk_cnt = p->chunk; sa.offsets = p->offsets;
   sa.gu_items = p->gu_items; sa.max_gu = static_cast<int>(p->max_gu);
   sa.dn_items = p->dn_items; sa.max_dn = static_cast<int>(p->max_dn);
   sa.item_counts = p->item_counts; sa.status = p->status;
-  route_scan_kernel<<<1, 1024, 0, s>>>(sa);
-  MOE_CUDA(cudaGetLastError(), "route_scan launch");
+  {
+    ProfScope ps(p, MOE_KERNEL_ROUTE_SCAN, s);
+    route_scan_kernel<<<1, 1024, 0, s>>>(sa);
+    MOE_CUDA(cudaGetLastError(), "route_scan launch");
+  }
   RouteScatterArgs ca;
   ca.T = T; ca.E = p->E; ca.k = p->k; ca.H = p->H;
   ca.ids = p->ids; ca.chunk_base = p->chunk; ca.perm = p->perm; ca.inv = p->inv;
   ca.x = x; ca.xt = p->xt; ca.xexp = p->xexp; ca.status = p->status;
-  route_scatter_kernel<<<nchunk, 256, 0, s>>>(ca);
-  MOE_CUDA(cudaGetLastError(), "route_scatter launch");
+  {
+    ProfScope ps(p, MOE_KERNEL_ROUTE_SCATTER, s);
+    route_scatter_kernel<<<nchunk, 256, 0, s>>>(ca);
+    MOE_CUDA(cudaGetLastError(), "route_scatter launch");
+  }
+  if (x) {
+    ProfScope ps(p, MOE_KERNEL_GATHER, s);
+    gather_kernel<<<tok_blocks, 256, 0, s>>>(ca);
+    MOE_CUDA(cudaGetLastError(), "gather launch");
+  }
   return MOE_OK;
 }
 
@@ -167,6 +211,7 @@ moe_status enqueue_layer(moe_plan_s *p, int T, const uint16_t *x, const float *l
     a.T = T; a.E = p->E; a.k = p->k; a.H = p->H; a.I = p->I; a.Is = p->Is;
     a.x = x; a.logits = logits; a.w = w; a.hbuf = p->hsmall; a.barrier = p->barrier;
     a.residual = residual; a.out = out; a.status = p->status;
+    ProfScope ps(p, MOE_KERNEL_SMALL_T, s);
     MOE_CUDA(launch_small_t(a, p->num_sms, s), "small-T kernel launch");
     return MOE_OK;
   }
@@ -183,15 +228,24 @@ moe_status enqueue_layer(moe_plan_s *p, int T, const uint16_t *x, const float *l
   g.items = p->gu_items;
   g.item_count = p->item_counts;
   g.max_items = static_cast<int>(max_gu_items(T, p->E, p->k, p->I, p->Is));
-  MOE_CUDA(launch_gemm_gate_up(g, p->num_sms, s), "gate/up GEMM launch");
+  {
+    ProfScope ps(p, MOE_KERNEL_GATE_UP, s);
+    MOE_CUDA(launch_gemm_gate_up(g, p->num_sms, s), "gate/up GEMM launch");
+  }
   g.items = p->dn_items;
   g.item_count = p->item_counts + 1;
   g.max_items = static_cast<int>(max_dn_items(T, p->E, p->k, p->H));
-  MOE_CUDA(launch_gemm_down(g, p->num_sms, s), "down GEMM launch");
+  {
+    ProfScope ps(p, MOE_KERNEL_DOWN, s);
+    MOE_CUDA(launch_gemm_down(g, p->num_sms, s), "down GEMM launch");
+  }
   CombineArgs c;
   c.T = T; c.k = p->k; c.H = p->H; c.R = T * p->k;
   c.inv = p->inv; c.y = p->y; c.xexp = p->xexp; c.residual = residual; c.out = out;
-  MOE_CUDA(launch_combine(c, s), "combine launch");
+  {
+    ProfScope ps(p, MOE_KERNEL_COMBINE, s);
+    MOE_CUDA(launch_combine(c, s), "combine launch");
+  }
   return MOE_OK;
 }
 
@@ -303,6 +357,7 @@ moe_status moe_plan_destroy(moe_plan_t *plan) {
   if (!plan) return fail(MOE_ERR_INVALID_ARG, "plan is NULL");
   cudaError_t err = cudaDeviceSynchronize();
   cudaError_t err2 = cudaFree(plan->ws);
+  for (cudaEvent_t e : plan->prof_events) cudaEventDestroy(e);
   delete plan;
   if (err != cudaSuccess) return cuda_fail(err, "synchronize before free");
   if (err2 != cudaSuccess) return cuda_fail(err2, "workspace cudaFree");
@@ -398,6 +453,45 @@ moe_status moe_route(moe_plan_t *plan, int T, const float *logits, int32_t *ids,
   if (offsets)
     MOE_CUDA(cudaMemcpyAsync(offsets, plan->offsets, (plan->E + 1) * 4, cudaMemcpyDeviceToDevice, s), "copy offsets");
   if (perm) MOE_CUDA(cudaMemcpyAsync(perm, plan->perm, R * 4, cudaMemcpyDeviceToDevice, s), "copy perm");
+  return MOE_OK;
+}
+
+moe_status moe_profile_enable(moe_plan_t *plan, int max_launches) {
+  g_last_error.clear();
+  if (!plan) return fail(MOE_ERR_INVALID_ARG, "plan is NULL");
+  if (max_launches < 0 || max_launches > (1 << 20)) return fail(MOE_ERR_INVALID_ARG, "max_launches out of range");
+  for (cudaEvent_t e : plan->prof_events) cudaEventDestroy(e);
+  plan->prof_events.clear();
+  plan->prof_kind.assign(max_launches, 0);
+  plan->prof_used = 0;
+  plan->prof_events.resize(2 * static_cast<size_t>(max_launches));
+  for (auto &e : plan->prof_events) {
+    cudaError_t err = cudaEventCreate(&e);
+    if (err != cudaSuccess) {
+      plan->prof_kind.clear();
+      return cuda_fail(err, "cudaEventCreate");
+    }
+  }
+  return MOE_OK;
+}
+
+moe_status moe_profile_read(moe_plan_t *plan, moe_stream_t stream, double *ms, int32_t *launches) {
+  g_last_error.clear();
+  if (!plan) return fail(MOE_ERR_INVALID_ARG, "plan is NULL");
+  MOE_CUDA(cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)), "stream synchronize");
+  double acc[MOE_KERNEL_COUNT] = {0};
+  int32_t cnt[MOE_KERNEL_COUNT] = {0};
+  for (int i = 0; i < plan->prof_used; ++i) {
+    float t = 0.f;
+    MOE_CUDA(cudaEventElapsedTime(&t, plan->prof_events[2 * i], plan->prof_events[2 * i + 1]), "event time");
+    acc[plan->prof_kind[i]] += t;
+    cnt[plan->prof_kind[i]] += 1;
+  }
+  plan->prof_used = 0;
+  for (int k = 0; k < MOE_KERNEL_COUNT; ++k) {
+    if (ms) ms[k] = acc[k];
+    if (launches) launches[k] = cnt[k];
+  }
   return MOE_OK;
 }
 

@@ -24,7 +24,7 @@ struct RouteScanArgs {
 struct RouteScatterArgs {
   int T, E, k, H;
   const int32_t *ids;         // [T*k]
-  const int32_t *chunk_base;  // [nchunk][E]
+  int32_t *chunk_base;        // [nchunk][E] bases in; zeroed on the way out
   int32_t *perm;              // [T*k]
   int32_t *inv;               // [T*k]
   const uint16_t *x;          // [T, H] bf16, or null (routing only)
@@ -89,6 +89,7 @@ __global__ void route_topk_kernel(int T, int E, int k, const float *__restrict__
                                   int32_t *__restrict__ chunk_cnt);
 __global__ void route_scan_kernel(RouteScanArgs a);
 __global__ void route_scatter_kernel(RouteScatterArgs a);
+__global__ void gather_kernel(RouteScatterArgs a);
 
 // host-side launchers (each returns the launch's cudaError_t)
 cudaError_t launch_gemm_gate_up(const GemmArgs &a, int num_sms, cudaStream_t s);

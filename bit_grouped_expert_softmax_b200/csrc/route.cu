@@ -22,25 +22,19 @@ __global__ void __launch_bounds__(256) route_topk_kernel(int T, int E, int k,
                                                          int32_t *__restrict__ ids,
                                                          float *__restrict__ wts,
                                                          int32_t *__restrict__ chunk_cnt) {
-  __shared__ int cnt[kMaxExperts];
-  const int chunk = blockIdx.x;
-  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
-  __syncthreads();
+  // one warp per token; the per-chunk expert histogram is built with integer
+  // atomics (order-independent) into chunk_cnt, which starts zeroed
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int t0 = chunk * kRouteChunk;
-  const int t1 = min(T, t0 + kRouteChunk);
-  for (int t = t0 + warp; t < t1; t += blockDim.x / 32) {
-    int id;
-    float w;
-    warp_topk(logits + static_cast<size_t>(t) * E, E, k, lane, id, w);
-    if (lane < k) {
-      ids[static_cast<size_t>(t) * k + lane] = id;
-      wts[static_cast<size_t>(t) * k + lane] = w;
-      atomicAdd(&cnt[id], 1);  // integer counts: order-independent
-    }
+  const int t = blockIdx.x * (blockDim.x >> 5) + warp;
+  if (t >= T) return;
+  int id;
+  float w;
+  warp_topk(logits + static_cast<size_t>(t) * E, E, k, lane, id, w);
+  if (lane < k) {
+    ids[static_cast<size_t>(t) * k + lane] = id;
+    wts[static_cast<size_t>(t) * k + lane] = w;
+    atomicAdd(&chunk_cnt[static_cast<size_t>(t / kRouteChunk) * E + id], 1);
   }
-  __syncthreads();
-  for (int e = threadIdx.x; e < E; e += blockDim.x) chunk_cnt[static_cast<size_t>(chunk) * E + e] = cnt[e];
 }
 
 // Single block. Turns per-chunk counts into per-chunk bases (in place), writes
@@ -51,18 +45,27 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(RouteScanArgs a) {
   __shared__ int gu_off[kMaxExperts + 2];
   __shared__ int dn_off[kMaxExperts + 2];
   __shared__ int warp_tot[3][32];
+  __shared__ int part[4][kMaxExperts];
   const int E = a.E;
   const int G = E + 1;  // routed experts plus the shared one
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    int run = 0;
-    for (int c = 0; c < a.nchunk; ++c) {
-      int32_t *p = a.chunk_cnt + static_cast<size_t>(c) * E + e;
-      const int v = *p;
-      *p = run;
-      run += v;
+  // each expert's column of per-chunk counts is split into four slices; the
+  // loads of a slice are issued in batches so they overlap
+  const int nq = (a.nchunk + 3) / 4;
+  const int e_t = threadIdx.x >> 2, q_t = threadIdx.x & 3;
+  const int c_lo = q_t * nq, c_hi = min(a.nchunk, c_lo + nq);
+  if (e_t < E) {
+    int sum = 0;
+    for (int c = c_lo; c < c_hi; c += 8) {
+      int v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = (c + u < c_hi) ? __ldcg(a.chunk_cnt + static_cast<size_t>(c + u) * E + e_t) : 0;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) sum += v[u];
     }
-    tot[e] = run;
+    part[q_t][e_t] = sum;
   }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) tot[e] = part[0][e] + part[1][e] + part[2][e] + part[3][e];
   __syncthreads();
   // exclusive scans over the groups, done by warp 0 with 9 values per lane (G <= 257)
   if (threadIdx.x < 32) {
@@ -109,8 +112,22 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(RouteScanArgs a) {
   }
   __syncthreads();
   for (int e = threadIdx.x; e <= E; e += blockDim.x) a.offsets[e] = (e < E) ? off[e] : a.T * a.k;
-  // per-chunk bases become absolute row positions
-  for (int i = threadIdx.x; i < a.nchunk * E; i += blockDim.x) a.chunk_cnt[i] += off[i % E];
+  // per-chunk counts become absolute row positions of each chunk's first entry
+  if (e_t < E) {
+    int base = off[e_t];
+    for (int q = 0; q < q_t; ++q) base += part[q][e_t];
+    for (int c = c_lo; c < c_hi; c += 8) {
+      int v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = (c + u < c_hi) ? __ldcg(a.chunk_cnt + static_cast<size_t>(c + u) * E + e_t) : 0;
+#pragma unroll
+      for (int u = 0; u < 8; ++u)
+        if (c + u < c_hi) {
+          a.chunk_cnt[static_cast<size_t>(c + u) * E + e_t] = base;
+          base += v[u];
+        }
+    }
+  }
   // work lists: group g's tiles are (n-tile, m-block) with the m-block fastest,
   // so neighbouring CTAs share the activation tile of one n-tile
   const int R = a.T * a.k;
@@ -140,87 +157,95 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(RouteScanArgs a) {
   }
 }
 
-// Stable scatter plus gather. One block per routing chunk of 32 tokens.
+// Stable scatter. One block per routing chunk of 32 tokens. The chunk's row of
+// bases is reset to zero afterwards, ready for the next routing's histogram.
 __global__ void __launch_bounds__(256) route_scatter_kernel(RouteScatterArgs a) {
   __shared__ int cnt[kMaxExperts];
-  __shared__ int pos_s[kRouteChunk * kMaxTopK];
   const int chunk = blockIdx.x, E = a.E, k = a.k, T = a.T;
-  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = a.chunk_base[static_cast<size_t>(chunk) * E + e];
+  int32_t *row = a.chunk_base + static_cast<size_t>(chunk) * E;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = __ldcg(row + e);
   __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) row[e] = 0;
   const int t0 = chunk * kRouteChunk, t1 = min(T, t0 + kRouteChunk);
   const int f0 = t0 * k, f1 = t1 * k;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (warp == 0) {
-    // flat order f = t*k + j is token-ascending; within a batch of 32 entries the
-    // rank among equal experts comes from match/popc, across batches from cnt[]
-    for (int fb = f0; fb < f1; fb += 32) {
-      const int f = fb + lane;
-      const bool valid = f < f1;
-      const unsigned active = __ballot_sync(0xffffffffu, valid);
-      if (valid) {
-        const int e = a.ids[f];
-        const unsigned peers = __match_any_sync(active, e);
-        const int rank = __popc(peers & ((1u << lane) - 1u));
-        const int base = cnt[e];
-        __syncwarp(active);
-        if (rank == 0) cnt[e] = base + __popc(peers);
-        const int pos = base + rank;
-        if (pos < 0 || pos >= T * k) {
-          report_error(a.status, kDevBounds, 20, static_cast<uint32_t>(pos));
-        } else {
-          a.perm[pos] = f;
-          a.inv[f] = pos;
-        }
-        pos_s[f - f0] = pos;
+  if (warp != 0) return;
+  // flat order f = t*k + j is token-ascending; within a batch of 32 entries the
+  // rank among equal experts comes from match/popc, across batches from cnt[]
+  for (int fb = f0; fb < f1; fb += 32) {
+    const int f = fb + lane;
+    const bool valid = f < f1;
+    const unsigned active = __ballot_sync(0xffffffffu, valid);
+    if (valid) {
+      const int e = a.ids[f];
+      const unsigned peers = __match_any_sync(active, e);
+      const int rank = __popc(peers & ((1u << lane) - 1u));
+      const int base = cnt[e];
+      __syncwarp(active);
+      if (rank == 0) cnt[e] = base + __popc(peers);
+      const int pos = base + rank;
+      if (pos < 0 || pos >= T * k) {
+        report_error(a.status, kDevBounds, 20, static_cast<uint32_t>(pos));
+      } else {
+        a.perm[pos] = f;
+        a.inv[f] = pos;
       }
-      __syncwarp();
+    }
+    __syncwarp();
+  }
+}
+
+// Gather: one warp per token. The row is scaled by a power of two 2^-e chosen
+// from its max |x| (exact in fp16 unless the row spans more than fp16's
+// range), converted to fp16 and written, in the K-permuted operand order, to
+// the token's k routed rows (positions from the scatter) and its shared-expert
+// row R + t.
+__global__ void __launch_bounds__(256) gather_kernel(RouteScatterArgs a) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * (blockDim.x >> 5) + warp;
+  if (t >= a.T) return;
+  const int H = a.H, k = a.k, R = a.T * k;
+  int rows[kMaxTopK];
+#pragma unroll
+  for (int j = 0; j < kMaxTopK; ++j) rows[j] = (j < k) ? a.inv[static_cast<size_t>(t) * k + j] : -1;
+  const uint4 *src = reinterpret_cast<const uint4 *>(a.x + static_cast<size_t>(t) * H);
+  const int nchunk8 = H / 8;
+  float amax = 0.f;
+  for (int c = lane; c < nchunk8; c += 32) {
+    const uint4 v = __ldg(src + c);
+    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      amax = fmaxf(amax, fabsf(__uint_as_float(w4[q] << 16)));
+      amax = fmaxf(amax, fabsf(__uint_as_float(w4[q] & 0xffff0000u)));
     }
   }
-  if (a.x == nullptr) return;
-  __syncthreads();
-  // gather: one warp per token; the row is scaled by a power of two 2^-e chosen
-  // from its max |x| (exact in fp16 unless the row spans more than fp16's range),
-  // converted to fp16 and written, in the K-permuted operand order, to the
-  // token's k routed rows and its shared-expert row
-  const int H = a.H, R = T * k;
-  const int nchunk8 = H / 8;
-  for (int t = t0 + warp; t < t1; t += blockDim.x / 32) {
-    const uint4 *src = reinterpret_cast<const uint4 *>(a.x + static_cast<size_t>(t) * H);
-    float amax = 0.f;
-    for (int c = lane; c < nchunk8; c += 32) {
-      const uint4 v = __ldg(src + c);
-      const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+  amax = warp_max(amax);
+  int ex = 0;
+  if (amax > 0.f && amax <= 3.0e38f) ex = min(max(ilogbf(amax) - 1, -100), 100);  // scaled max in [2, 4)
+  const float scale = exp2f(static_cast<float>(-ex));
+  if (lane == 0) a.xexp[t] = ex;
+  for (int c = lane; c < nchunk8; c += 32) {
+    const uint4 v = __ldg(src + c);
+    const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+    __half hv[8];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        amax = fmaxf(amax, fabsf(__uint_as_float(w4[q] << 16)));
-        amax = fmaxf(amax, fabsf(__uint_as_float(w4[q] & 0xffff0000u)));
+    for (int q = 0; q < 4; ++q) {
+      hv[2 * q] = __float2half_rn(__uint_as_float(w4[q] << 16) * scale);
+      hv[2 * q + 1] = __float2half_rn(__uint_as_float(w4[q] & 0xffff0000u) * scale);
+    }
+    uint4 o;
+    uint32_t *op = reinterpret_cast<uint32_t *>(&o);
+#pragma unroll
+    for (int s = 0; s < 8; s += 2) op[s / 2] = pack_half2(hv[kperm_src(s)], hv[kperm_src(s + 1)]);
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j) {
+      if (j < k) {
+        const int row = rows[j];
+        if (row >= 0 && row < R) reinterpret_cast<uint4 *>(a.xt + static_cast<size_t>(row) * H)[c] = o;
       }
     }
-    amax = warp_max(amax);
-    int ex = 0;
-    if (amax > 0.f && amax <= 3.0e38f) ex = min(max(ilogbf(amax) - 1, -100), 100);  // scaled max in [2, 4)
-    const float scale = exp2f(static_cast<float>(-ex));
-    if (lane == 0) a.xexp[t] = ex;
-    for (int c = lane; c < nchunk8; c += 32) {
-      const uint4 v = __ldg(src + c);
-      const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-      __half hv[8];
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        hv[2 * q] = __float2half_rn(__uint_as_float(w4[q] << 16) * scale);
-        hv[2 * q + 1] = __float2half_rn(__uint_as_float(w4[q] & 0xffff0000u) * scale);
-      }
-      uint4 o;
-      uint32_t *op = reinterpret_cast<uint32_t *>(&o);
-#pragma unroll
-      for (int s = 0; s < 8; s += 2) op[s / 2] = pack_half2(hv[kperm_src(s)], hv[kperm_src(s + 1)]);
-      for (int j = 0; j < k; ++j) {
-        const int row = pos_s[(t - t0) * k + j];
-        if (row >= 0 && row < R)
-          reinterpret_cast<uint4 *>(a.xt + static_cast<size_t>(row) * H)[c] = o;
-      }
-      reinterpret_cast<uint4 *>(a.xt + static_cast<size_t>(R + t) * H)[c] = o;
-    }
+    reinterpret_cast<uint4 *>(a.xt + static_cast<size_t>(R + t) * H)[c] = o;
   }
 }
 

@@ -169,6 +169,29 @@ moe_status moe_route(moe_plan_t *plan, int T, const float *logits, int32_t *ids,
  */
 moe_status moe_status_sync(moe_plan_t *plan, moe_stream_t stream);
 
+/*
+ * Per-kernel timing. While enabled, every kernel the plan enqueues is
+ * bracketed by two CUDA events recorded on the launching stream (up to
+ * max_launches launches; later ones are not recorded). moe_profile_read waits
+ * for the stream, adds up the elapsed times per kernel kind into
+ * ms[MOE_KERNEL_COUNT] and launches[MOE_KERNEL_COUNT] (either may be NULL)
+ * and starts a new recording window. max_launches = 0 disables recording.
+ * Not for use while the stream is being captured into a CUDA graph.
+ */
+enum {
+  MOE_KERNEL_ROUTE_TOPK = 0,
+  MOE_KERNEL_ROUTE_SCAN = 1,
+  MOE_KERNEL_ROUTE_SCATTER = 2,
+  MOE_KERNEL_GATHER = 3,
+  MOE_KERNEL_GATE_UP = 4,
+  MOE_KERNEL_DOWN = 5,
+  MOE_KERNEL_COMBINE = 6,
+  MOE_KERNEL_SMALL_T = 7,
+  MOE_KERNEL_COUNT = 8
+};
+moe_status moe_profile_enable(moe_plan_t *plan, int max_launches);
+moe_status moe_profile_read(moe_plan_t *plan, moe_stream_t stream, double *ms, int32_t *launches);
+
 /* Message of the last failed call on this thread ("" if none). */
 const char *moe_last_error(void);
 
