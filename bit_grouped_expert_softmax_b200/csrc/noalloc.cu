@@ -1,0 +1,118 @@
+// noalloc.cu -- the small-T layer without any device allocation.
+//
+// Some callers cannot call cudaMalloc: code that runs inside an allocator
+// callback or a custom memory pool that owns all device memory, embedded
+// runtimes that pre-reserve every byte at start-up, or hosts where the
+// allocation API is not reachable from the thread that issues work. For them,
+// moe_forward_small_t_noalloc runs the fused small-T kernel (batches of at
+// most 8 tokens) with its scratch memory -- the per-token SwiGLU outputs, the
+// grid-barrier words and the device status word -- taken from one file-scope
+// __device__ array instead of a plan's workspace. The caller still passes all
+// inputs and outputs.
+//
+// The array is created when the library's module is loaded on a device and
+// stays until the process exits, on every GPU that loads the library.
+#include <mutex>
+
+#include "../../include/moe_b200.h"
+#include "kernels.cuh"
+
+namespace moe {
+size_t small_t_smem_bytes(int T, int H, int k, int I, int Is);
+void set_last_error(const char *msg);  // the message moe_last_error() returns on this thread
+}
+
+using namespace moe;
+
+namespace {
+
+constexpr size_t kStaticScratchBytes = 512 * 1024;  // stated maximum
+constexpr size_t kHeaderBytes = 256;                // barrier words + status word
+constexpr int kMaxDevices = 64;
+
+// [0, 16): grid barrier {count, generation}; [16, 32): DevStatus;
+// [256, kStaticScratchBytes): fp32 SwiGLU outputs, T * (top_k + 1) * max(I, Is)
+static __device__ __align__(256) unsigned char g_small_t_scratch[kStaticScratchBytes];
+
+struct DeviceSlot {
+  std::once_flag once;
+  cudaError_t err = cudaSuccess;
+  unsigned char *ptr = nullptr;  // device address of g_small_t_scratch on this device
+  int num_sms = 0;
+};
+DeviceSlot g_slots[kMaxDevices];
+
+moe_status fail(moe_status st, const char *msg) {
+  set_last_error(msg);
+  return st;
+}
+
+}  // namespace
+
+extern "C" moe_status moe_forward_small_t_noalloc(int T, int hidden, int n_experts, int top_k, int inter,
+                                                  int shared_inter, const void *x_bf16, const float *router_logits,
+                                                  const uint32_t *packed_w, const void *scales, const void *biases,
+                                                  const uint32_t *shared_packed_w, const void *shared_scales,
+                                                  const void *shared_biases, void *out_bf16, void *status_out,
+                                                  moe_stream_t stream) {
+  set_last_error("");
+  if (T < 0 || T > kSmallT) return fail(MOE_ERR_INVALID_ARG, "T must be in [0, 8]");
+  if (hidden < 128 || hidden % 128 || hidden > 16384 || inter < 128 || inter % 128 || inter > 8192 ||
+      shared_inter < 128 || shared_inter % 128 || shared_inter > 8192)
+    return fail(MOE_ERR_INVALID_ARG, "hidden, inter and shared_inter must be positive multiples of 128");
+  if (n_experts < 1 || n_experts > kMaxExperts || top_k < 1 || top_k > n_experts || top_k > kMaxTopK)
+    return fail(MOE_ERR_INVALID_ARG, "need 1 <= top_k <= min(n_experts, 16) and n_experts <= 256");
+  const size_t imax = static_cast<size_t>(inter > shared_inter ? inter : shared_inter);
+  const size_t h_bytes = static_cast<size_t>(kSmallT) * (top_k + 1) * imax * sizeof(float);
+  if (kHeaderBytes + h_bytes > kStaticScratchBytes)
+    return fail(MOE_ERR_UNSUPPORTED, "8 * (top_k + 1) * max(inter, shared_inter) * 4 bytes exceeds the 512 KiB "
+                                     "static scratch");
+  if (small_t_smem_bytes(T, hidden, top_k, inter, shared_inter) > 200 * 1024)
+    return fail(MOE_ERR_UNSUPPORTED, "layer too large for the small-T kernel's shared memory");
+  if (T == 0) return MOE_OK;
+  const void *ptrs[10] = {x_bf16, router_logits, packed_w, scales, biases, shared_packed_w, shared_scales,
+                          shared_biases, out_bf16, nullptr};
+  for (int i = 0; i < 9; ++i)
+    if (!ptrs[i] || (reinterpret_cast<uintptr_t>(ptrs[i]) & 15u))
+      return fail(MOE_ERR_INVALID_ARG, "tensor pointers must be non-NULL and 16-byte aligned");
+  if (x_bf16 == out_bf16) return fail(MOE_ERR_INVALID_ARG, "out must not alias x");
+
+  int dev = 0;
+  cudaError_t err = cudaGetDevice(&dev);
+  if (err != cudaSuccess) return fail(MOE_ERR_NO_DEVICE, "no current CUDA device");
+  if (dev < 0 || dev >= kMaxDevices) return fail(MOE_ERR_UNSUPPORTED, "device ordinal above 63");
+  DeviceSlot &slot = g_slots[dev];
+  // once per device, with that device current: the array's device address
+  std::call_once(slot.once, [&slot, dev]() {
+    slot.err = cudaGetSymbolAddress(reinterpret_cast<void **>(&slot.ptr), g_small_t_scratch);
+    if (slot.err == cudaSuccess) slot.err = cudaDeviceGetAttribute(&slot.num_sms, cudaDevAttrMultiProcessorCount, dev);
+  });
+  if (slot.err != cudaSuccess || !slot.ptr) return fail(MOE_ERR_CUDA, "cudaGetSymbolAddress of the static scratch failed");
+
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  // the array keeps the previous call's contents: reset the barrier and status words
+  err = cudaMemsetAsync(slot.ptr, 0, kHeaderBytes, s);
+  if (err != cudaSuccess) return fail(MOE_ERR_CUDA, "clearing the static scratch header failed");
+  SmallTArgs a;
+  a.T = T; a.E = n_experts; a.k = top_k; a.H = hidden; a.I = inter; a.Is = shared_inter;
+  a.x = static_cast<const uint16_t *>(x_bf16);
+  a.logits = router_logits;
+  a.w.packed = packed_w;
+  a.w.scales = static_cast<const uint16_t *>(scales);
+  a.w.biases = static_cast<const uint16_t *>(biases);
+  a.w.sh_packed = shared_packed_w;
+  a.w.sh_scales = static_cast<const uint16_t *>(shared_scales);
+  a.w.sh_biases = static_cast<const uint16_t *>(shared_biases);
+  a.barrier = reinterpret_cast<uint32_t *>(slot.ptr);
+  a.status = reinterpret_cast<DevStatus *>(slot.ptr + 16);
+  a.hbuf = reinterpret_cast<float *>(slot.ptr + kHeaderBytes);
+  a.residual = nullptr;
+  a.out = static_cast<uint16_t *>(out_bf16);
+  err = launch_small_t(a, slot.num_sms, s);
+  if (err != cudaSuccess) return fail(MOE_ERR_CUDA, "small-T kernel launch failed");
+  if (status_out) {
+    err = cudaMemcpyAsync(status_out, slot.ptr + 16, sizeof(DevStatus), cudaMemcpyDeviceToDevice, s);
+    if (err != cudaSuccess) return fail(MOE_ERR_CUDA, "copying the device status failed");
+  }
+  return MOE_OK;
+}

@@ -192,6 +192,36 @@ enum {
 moe_status moe_profile_enable(moe_plan_t *plan, int max_launches);
 moe_status moe_profile_read(moe_plan_t *plan, moe_stream_t stream, double *ms, int32_t *launches);
 
+/*
+ * The small-T layer (0 <= T <= 8 tokens) without any device allocation.
+ * The paper has no counterpart to this call; it exists for callers that
+ * cannot call cudaMalloc (code running inside an allocator or memory-pool
+ * callback, runtimes that reserve all device memory up front), and so cannot
+ * create a plan. Its scratch memory (SwiGLU outputs, grid-barrier words,
+ * status word) lives in one static __device__ array of 512 KiB inside the
+ * library, which every GPU that loads the library holds until the process
+ * exits; the caller passes only inputs and outputs, as for moe_forward.
+ *   Sizes: as moe_plan, plus 8 * (top_k + 1) * max(inter, shared_inter) * 4
+ *   bytes must fit in 512 KiB - 256 bytes; larger layers get
+ *   MOE_ERR_UNSUPPORTED, T > 8 gets MOE_ERR_INVALID_ARG.
+ *   status_out: optional device pointer to 16 bytes that receive the device
+ *   status word of this call ({code, site, detail, 0}; code 0 = OK).
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before capturing
+ * the stream into a CUDA graph. Each call clears the barrier and status words
+ * on the stream and calls no cudaMalloc, cudaFree or allocating library
+ * routine. All calls share the one array, so calls that overlap on the GPU
+ * (different streams, or several devices' work mixed up in one process is
+ * fine -- each device has its own copy) race: serialise them on one stream.
+ */
+moe_status moe_forward_small_t_noalloc(int T, int hidden, int n_experts, int top_k, int inter,
+                                       int shared_inter, const void *x_bf16,
+                                       const float *router_logits, const uint32_t *packed_w,
+                                       const void *scales, const void *biases,
+                                       const uint32_t *shared_packed_w, const void *shared_scales,
+                                       const void *shared_biases, void *out_bf16, void *status_out,
+                                       moe_stream_t stream);
+
 /* Message of the last failed call on this thread ("" if none). */
 const char *moe_last_error(void);
 
