@@ -210,9 +210,9 @@ moe_status moe_profile_read(moe_plan_t *plan, moe_stream_t stream, double *ms, i
  * device, with that device current); make that first call before capturing
  * the stream into a CUDA graph. Each call clears the barrier and status words
  * on the stream and calls no cudaMalloc, cudaFree or allocating library
- * routine. All calls share the one array, so calls that overlap on the GPU
- * (different streams, or several devices' work mixed up in one process is
- * fine -- each device has its own copy) race: serialise them on one stream.
+ * routine. All calls on one device share that device's copy of the array,
+ * so calls that overlap on the GPU (for example on two streams) race:
+ * serialise them on one stream.
  */
 moe_status moe_forward_small_t_noalloc(int T, int hidden, int n_experts, int top_k, int inter,
                                        int shared_inter, const void *x_bf16,
