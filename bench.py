@@ -149,6 +149,8 @@ def run_gpu(args, rank, world, local_rank):
         touched = max(rf["weight_bytes"], 1)
         n_rep = int(min(32, max(2, -(-4 * l2 // touched))))
         n_rep = int(min(n_rep, max(2, (40 << 30) // layer_bytes)))
+        if args.replicas:
+            n_rep = args.replicas
         reps = [base] + [api.DeviceLayer(*[t.clone() for t in base.args()]) for _ in range(n_rep - 1)]
         x = torch.from_numpy(inp.x.view(np.int16)).to(dev)
         logits = torch.from_numpy(inp.logits).to(dev)
@@ -317,6 +319,8 @@ def main():
     ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "zipf", "tiny"])
     ap.add_argument("--no-extra", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--replicas", type=int, default=0,
+                    help="weight replicas to rotate over (default: enough to exceed 4x L2); for profiling runs")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 

@@ -9,7 +9,7 @@
 #include <string>
 #include <vector>
 
-#include "../../include/moe_b200.h"
+#include "moe_b200.h"
 #include "kernels.cuh"
 
 namespace moe {
@@ -81,6 +81,8 @@ struct moe_plan_s {
   int32_t *offsets;
   int32_t *perm;
   int32_t *inv;
+  int32_t *row_exp;
+  float *row_w;
   WorkItem *gu_items;
   WorkItem *dn_items;
   int32_t *item_counts;
@@ -188,6 +190,7 @@ moe_status enqueue_routing(moe_plan_s *p, int T, const float *logits, const uint
   ca.T = T; ca.E = p->E; ca.k = p->k; ca.H = p->H;
   ca.ids = p->ids; ca.chunk_base = p->chunk; ca.perm = p->perm; ca.inv = p->inv;
   ca.x = x; ca.xt = p->xt; ca.xexp = p->xexp; ca.status = p->status;
+  ca.wts = p->wts; ca.row_exp = p->row_exp; ca.row_w = p->row_w;
   {
     ProfScope ps(p, MOE_KERNEL_ROUTE_SCATTER, s);
     route_scatter_kernel<<<nchunk, 256, 0, s>>>(ca);
@@ -222,6 +225,7 @@ moe_status enqueue_layer(moe_plan_s *p, int T, const uint16_t *x, const float *l
   g.w = w; g.xt = p->xt; g.h = p->h;
   g.h_shared_off = static_cast<int64_t>(p->T_max) * p->k * p->I;
   g.y = p->y; g.perm = p->perm; g.wts = p->wts; g.xexp = p->xexp; g.status = p->status;
+  g.row_exp = p->row_exp; g.row_w = p->row_w;
   g.xt_rows = static_cast<int64_t>(p->T_max) * (p->k + 1);
   g.h_rows = static_cast<int64_t>(p->T_max) * p->k;
   g.hs_rows = p->T_max;
@@ -295,6 +299,8 @@ moe_status moe_plan(int T_max, int hidden, int n_experts, int top_k, int inter, 
       (E + 1) * 4,                           // offsets
       R * 4,                                 // perm
       R * 4,                                 // inv
+      (R + T) * 4,                           // row_exp
+      (R + T) * 4,                           // row_w
       static_cast<size_t>(p->max_gu) * sizeof(WorkItem),
       static_cast<size_t>(p->max_dn) * sizeof(WorkItem),
       16,                                    // item counts
@@ -329,6 +335,8 @@ moe_status moe_plan(int T_max, int hidden, int n_experts, int top_k, int inter, 
   p->offsets = reinterpret_cast<int32_t *>(b + offs[i++]);
   p->perm = reinterpret_cast<int32_t *>(b + offs[i++]);
   p->inv = reinterpret_cast<int32_t *>(b + offs[i++]);
+  p->row_exp = reinterpret_cast<int32_t *>(b + offs[i++]);
+  p->row_w = reinterpret_cast<float *>(b + offs[i++]);
   p->gu_items = reinterpret_cast<WorkItem *>(b + offs[i++]);
   p->dn_items = reinterpret_cast<WorkItem *>(b + offs[i++]);
   p->item_counts = reinterpret_cast<int32_t *>(b + offs[i++]);

@@ -30,6 +30,9 @@ struct RouteScatterArgs {
   const uint16_t *x;          // [T, H] bf16, or null (routing only)
   __half *xt;                 // [T*k + T, H] gathered fp16 rows
   int32_t *xexp;              // [T] power-of-two exponent of each token's row scale
+  const float *wts;           // [T*k] routing weights by flat index
+  int32_t *row_exp;           // [T*k + T] exponent of the token of each gathered row
+  float *row_w;               // [T*k + T] routing weight of each row (1 for shared rows)
   DevStatus *status;
 };
 
@@ -54,6 +57,8 @@ struct GemmArgs {
   const int32_t *perm;      // [R] row -> flat index t*k+j
   const float *wts;         // [T*k] routing weights by flat index
   const int32_t *xexp;      // [T]
+  const int32_t *row_exp;   // [R+T] exponent of each row's token
+  const float *row_w;       // [R+T] routing weight of each row (1 for shared rows)
   const WorkItem *items;
   const int32_t *item_count;
   int max_items;

@@ -14,7 +14,7 @@
 // stays until the process exits, on every GPU that loads the library.
 #include <mutex>
 
-#include "../../include/moe_b200.h"
+#include "moe_b200.h"
 #include "kernels.cuh"
 
 namespace moe {

@@ -189,6 +189,7 @@ __global__ void __launch_bounds__(256) route_scatter_kernel(RouteScatterArgs a) 
       } else {
         a.perm[pos] = f;
         a.inv[f] = pos;
+        a.row_w[pos] = a.wts[f];
       }
     }
     __syncwarp();
@@ -225,6 +226,14 @@ __global__ void __launch_bounds__(256) gather_kernel(RouteScatterArgs a) {
   if (amax > 0.f && amax <= 3.0e38f) ex = min(max(ilogbf(amax) - 1, -100), 100);  // scaled max in [2, 4)
   const float scale = exp2f(static_cast<float>(-ex));
   if (lane == 0) a.xexp[t] = ex;
+  // per-row epilogue factors of the token's k + 1 rows
+#pragma unroll
+  for (int j = 0; j < kMaxTopK; ++j)
+    if (j < k && lane == j && rows[j] >= 0 && rows[j] < R) a.row_exp[rows[j]] = ex;
+  if (lane == 0) {
+    a.row_exp[R + t] = ex;
+    a.row_w[R + t] = 1.0f;
+  }
   for (int c = lane; c < nchunk8; c += 32) {
     const uint4 v = __ldg(src + c);
     const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
