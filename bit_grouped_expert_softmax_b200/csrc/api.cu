@@ -133,8 +133,7 @@ moe_status check_weights(const moe_plan_s *p, const void *packed, const void *sc
 
 bool use_small_t(const moe_plan_s *p, int T) {
   if (p->flags & MOE_FLAG_FORCE_GROUPED) return false;
-  if (T > kSmallT) return false;
-  return small_t_smem_bytes(T, p->H, p->k, p->I, p->Is) <= 200 * 1024;
+  return small_t_fits(T, p->H, p->k, p->I, p->Is, p->num_sms);
 }
 
 LayerWeights make_weights(const void *packed, const void *scales, const void *biases, const void *spacked,
@@ -208,7 +207,7 @@ moe_status enqueue_layer(moe_plan_s *p, int T, const uint16_t *x, const float *l
                          const uint16_t *residual, uint16_t *out, cudaStream_t s) {
   if (T == 0) return MOE_OK;
   if (use_small_t(p, T) || (p->flags & MOE_FLAG_FORCE_SMALL_T)) {
-    if (T > kSmallT || small_t_smem_bytes(T, p->H, p->k, p->I, p->Is) > 200 * 1024)
+    if (!small_t_fits(T, p->H, p->k, p->I, p->Is, p->num_sms))
       return fail(MOE_ERR_UNSUPPORTED, "small-T path needs T <= %d and a small enough layer", kSmallT);
     SmallTArgs a;
     a.T = T; a.E = p->E; a.k = p->k; a.H = p->H; a.I = p->I; a.Is = p->Is;

@@ -67,8 +67,6 @@ extern "C" moe_status moe_forward_small_t_noalloc(int T, int hidden, int n_exper
   if (kHeaderBytes + h_bytes > kStaticScratchBytes)
     return fail(MOE_ERR_UNSUPPORTED, "8 * (top_k + 1) * max(inter, shared_inter) * 4 bytes exceeds the 512 KiB "
                                      "static scratch");
-  if (small_t_smem_bytes(T, hidden, top_k, inter, shared_inter) > 200 * 1024)
-    return fail(MOE_ERR_UNSUPPORTED, "layer too large for the small-T kernel's shared memory");
   if (T == 0) return MOE_OK;
   const void *ptrs[10] = {x_bf16, router_logits, packed_w, scales, biases, shared_packed_w, shared_scales,
                           shared_biases, out_bf16, nullptr};
@@ -88,6 +86,8 @@ extern "C" moe_status moe_forward_small_t_noalloc(int T, int hidden, int n_exper
     if (slot.err == cudaSuccess) slot.err = cudaDeviceGetAttribute(&slot.num_sms, cudaDevAttrMultiProcessorCount, dev);
   });
   if (slot.err != cudaSuccess || !slot.ptr) return fail(MOE_ERR_CUDA, "cudaGetSymbolAddress of the static scratch failed");
+  if (!small_t_fits(T, hidden, top_k, inter, shared_inter, slot.num_sms))
+    return fail(MOE_ERR_UNSUPPORTED, "layer too large for the small-T kernel");
 
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   // the array keeps the previous call's contents: reset the barrier and status words

@@ -2,80 +2,220 @@
 //
 // Batch-1 decode has almost no weight reuse, so memory bandwidth sets the
 // ceiling (aioga.com record of the Lily report, article body paragraph 6).
-// One persistent kernel, one CTA per SM, does the whole layer:
-//   phase 0  every CTA routes the (<= 8) tokens itself (same result everywhere),
-//            builds the list of distinct experts used, stages x in shared memory
-//   phase 1  gate/up rows of the used experts, one row pair per warp at a time,
-//            128-bit coalesced loads of the packed words; each group of 64 uses
-//            sum_i x_i (q_i s + b) = s * sum_i x_i q_i + b * sum_i x_i in fp32;
-//            h = silu(gate) * up goes to a small fp32 scratch buffer
+// One persistent cooperative kernel, one CTA per SM, does the whole layer so
+// that every weight byte it needs is requested as early as possible:
+//
+//   phase 0  every CTA routes the (<= 8) tokens itself (same result in every
+//            CTA), lists the distinct experts used, stages the tokens as fp16
+//            (scaled by a power of two per token) in the operand order below,
+//            and requests -- with bulk asynchronous copies into shared memory --
+//            the gate/up row blocks and the down-projection rows it will need;
+//            the shared expert's first block is requested before routing ends
+//   phase 1  gate/up: each 16-row block of an expert is split along K over
+//            several warps; tensor-core mma.sync m16n8k16 with A = dequantised
+//            weights (fp16 q*scale+bias, as in the grouped GEMM) and B = the
+//            tokens (N = 8 covers every token at once); partial sums reduced in
+//            a fixed order, then h = silu(gate) * up goes to a small scratch
 //   barrier  bounded grid barrier (the launch is cooperative)
-//   phase 2  down rows: each warp owns output columns n and sums, per token,
-//            w_j * y_j over j = 0..k-1 then the shared expert, in that fixed order
+//   phase 2  down: each CTA owns 16 output features; its warps take the used
+//            experts, weighting each token's result by its routing weight; the
+//            warps' results are summed in a fixed order and rounded once
+//
+// Operand order along K: packed word W holds elements 8W..8W+7; the fp16
+// operands store them at positions 8W + s in the pair order (0,4),(1,5),(2,6),
+// (3,7) that the int4 conversion produces. Within each block of 16 words,
+// thread c of an mma quad takes words 4c..4c+3, one per mma pair; both
+// operands index the same word, so the products are those of the plain dot
+// product.
+#include <algorithm>
+
 #include "kernels.cuh"
+#include "sm100.cuh"
 #include "topk.cuh"
 
 namespace moe {
 
 namespace {
 
+using namespace sm100;
+
 constexpr int kSTWarps = 16;
 constexpr int kSTThreads = kSTWarps * 32;
-constexpr int kXPitch = 68;  // floats per 64-element group of x in shared memory (padded)
+constexpr int kRowBlock = 16;  // weight rows per mma tile
+constexpr int kXPad = 32;      // fp16 padding per staged token row (bank spread)
+constexpr int kMaxU = kSmallT * kMaxTopK + 1;
 
 struct SmallTShared {
   int ids[kSmallT][kMaxTopK];
   float wt[kSmallT][kMaxTopK];
-  int ulist[kSmallT * kMaxTopK + 1];
-  uint32_t umask[kSmallT * kMaxTopK + 1];
-  int8_t uslot[kSmallT * kMaxTopK + 1][kSmallT];  // slot j of expert u in token t (-1: unused)
+  int xexp[kSmallT];                   // max |x| bits, then the token's exponent
+  uint32_t bitmap[kMaxExperts / 32];   // experts used by any token
+  int ulist[kMaxU];                    // distinct experts, ascending, then the shared one (E)
+  uint32_t umask[kMaxU];               // tokens routed to each
+  int8_t uslot[kMaxU][kSmallT];        // slot j of expert u in token t (-1: none; k: shared)
   int nU;
   int ok;
+  int abort;
 };
 
-__device__ __forceinline__ float code_f(uint32_t w, int j) {
-  // exact float of the 4-bit code j of w: 2^23 + q as a float, minus 2^23
-  return __uint_as_float(0x4B000000u | ((w >> (4 * j)) & 0xFu)) - 8388608.0f;
+// Per-launch layout of the dynamic shared memory.
+struct StLayout {
+  int Imax, kw, ks;   // max intermediate, K per warp and warps per row block in phase 1
+  int nb, nd;         // stages of the phase-1 and phase-2 rings
+  size_t x_off, red_off, b_off, d_off, bar_off, bytes;
+  size_t b_stage, d_stage;
+};
+
+__host__ __device__ inline StLayout st_layout(int H, int I, int Is, int T, int k) {
+  StLayout L;
+  L.Imax = I > Is ? I : Is;
+  L.ks = H / kGroup < 8 ? H / kGroup : 8;
+  L.kw = H / L.ks;
+  L.b_stage = static_cast<size_t>(2) * kRowBlock * (H / 2) + static_cast<size_t>(4) * kRowBlock * (H / kGroup) * 2;
+  L.d_stage = static_cast<size_t>(kRowBlock) * (L.Imax / 2) + static_cast<size_t>(2) * kRowBlock * (L.Imax / kGroup) * 2;
+  L.x_off = 0;
+  const size_t x_bytes = static_cast<size_t>(kSmallT) * (H + kXPad) * 2;
+  L.red_off = (x_bytes + 127) / 128 * 128;
+  const size_t red_bytes = static_cast<size_t>(kSTThreads) * 8 * 4;
+  L.b_off = L.red_off + red_bytes;
+  const size_t budget = 220 * 1024;
+  const size_t h_bytes = static_cast<size_t>(T) * (k + 1) * L.Imax * 2;  // phase-2 copy of h (in the B ring)
+  // phase-1 ring: the most stages (up to 4) that still leave the down ring one
+  // stage per used expert (or at least 8); the B ring must also hold h later
+  const int want_d = T * k + 1;
+  L.nb = 0;
+  L.nd = 0;
+  for (int nb = 4; nb >= 2; --nb) {
+    const size_t used = L.b_off + nb * L.b_stage + 512;
+    if (used >= budget || nb * L.b_stage < h_bytes) continue;
+    int nd = static_cast<int>((budget - used) / L.d_stage);
+    nd = nd < want_d ? nd : want_d;
+    if (nd >= (want_d < 8 ? want_d : 8) || nb == 2) {
+      L.nb = nb;
+      L.nd = nd;
+      break;
+    }
+  }
+  L.d_off = L.b_off + L.nb * L.b_stage;
+  L.bar_off = L.d_off + L.nd * L.d_stage;
+  L.bytes = L.bar_off + 2 * (L.nb + L.nd) * 8 + 16;
+  return L;
 }
 
-// sum over the 8 codes of a word of q_j * x[j]
-__device__ __forceinline__ float dot8(uint32_t w, const float *x) {
-  float acc = 0.f;
-#pragma unroll
-  for (int j = 0; j < 8; ++j) acc = fmaf(code_f(w, j), x[j], acc);
-  return acc;
+// Bounded wait on an mbarrier phase; on timeout or abort returns false.
+__device__ __forceinline__ bool st_wait(uint64_t *bar, uint32_t parity, volatile int *abort, DevStatus *st,
+                                        uint32_t site) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort) return false;
+    if (global_ns() - t0 > kWaitBudgetNs) {
+      *abort = 1;
+      report_error(st, kDevTimeout, site, blockIdx.x);
+      return false;
+    }
+  }
 }
 
-// Grid barrier on {count, generation}; returns false if the wait ran out.
+__device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+      "{%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Grid barrier on {count, generation} with release/acquire atomics; returns
+// false if the wait ran out. The last CTA to arrive resets the count and bumps
+// the generation.
 __device__ bool grid_barrier(uint32_t *bar, DevStatus *st, int *ok_flag) {
   __syncthreads();
   if (threadIdx.x == 0) {
-    volatile uint32_t *vgen = bar + 1;
-    const uint32_t gen = *vgen;
-    __threadfence();
-    const uint32_t arrived = atomicAdd(bar, 1u);
+    uint32_t gen;
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(gen) : "l"(bar + 1) : "memory");
+    uint32_t arrived;
+    asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;" : "=r"(arrived) : "l"(bar) : "memory");
+    int ok = 1;
     if (arrived == gridDim.x - 1) {
-      atomicExch(bar, 0u);
-      __threadfence();
-      atomicAdd(bar + 1, 1u);
-      *ok_flag = 1;
+      asm volatile("st.relaxed.gpu.global.u32 [%0], 0;" ::"l"(bar) : "memory");
+      asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(bar + 1) : "memory");
     } else {
       const unsigned long long t0 = global_ns();
-      int ok = 1;
       unsigned it = 0;
-      while (*vgen == gen) {
-        if ((++it & 1023u) == 0 && global_ns() - t0 > kWaitBudgetNs) {
+      while (true) {
+        uint32_t g;
+        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(g) : "l"(bar + 1) : "memory");
+        if (g != gen) break;
+        __nanosleep(32);
+        if ((++it & 63u) == 0 && global_ns() - t0 > kWaitBudgetNs) {
           report_error(st, kDevTimeout, 30, blockIdx.x);
           ok = 0;
           break;
         }
       }
-      *ok_flag = ok;
     }
-    __threadfence();
+    *ok_flag = ok;
   }
   __syncthreads();
   return *ok_flag != 0;
+}
+
+// Weight pointers of one expert id (E = the shared expert).
+struct ExpertPtrs {
+  const uint32_t *packed;
+  const uint16_t *scales, *biases;
+  int Iu;
+};
+
+__device__ __forceinline__ ExpertPtrs expert_ptrs(const SmallTArgs &a, int e) {
+  ExpertPtrs p;
+  if (e == a.E) {
+    p.packed = a.w.sh_packed;
+    p.scales = a.w.sh_scales;
+    p.biases = a.w.sh_biases;
+    p.Iu = a.Is;
+  } else {
+    p.packed = a.w.packed + static_cast<size_t>(e) * 3 * a.I * a.H / 8;
+    p.scales = a.w.scales + static_cast<size_t>(e) * 3 * a.I * a.H / kGroup;
+    p.biases = a.w.biases + static_cast<size_t>(e) * 3 * a.I * a.H / kGroup;
+    p.Iu = a.I;
+  }
+  return p;
+}
+
+// 8 bf16 values -> 8 fp16 values scaled by 2^-ex, in operand order
+__device__ __forceinline__ uint4 x_scaled_fp16(uint4 v, int ex) {
+  const float scale = __int_as_float((127 - ex) << 23);  // 2^-ex, |ex| <= 100
+  const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+  __half hv[8];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    hv[2 * q] = __float2half_rn(__uint_as_float(w4[q] << 16) * scale);
+    hv[2 * q + 1] = __float2half_rn(__uint_as_float(w4[q] & 0xffff0000u) * scale);
+  }
+  uint4 o;
+  uint32_t *op = reinterpret_cast<uint32_t *>(&o);
+#pragma unroll
+  for (int s2 = 0; s2 < 8; s2 += 2) op[s2 / 2] = pack_half2(hv[kperm_src(s2)], hv[kperm_src(s2 + 1)]);
+  return o;
+}
+
+__device__ __forceinline__ float bf16x8_absmax(uint4 v) {
+  const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+  float m = 0.f;
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    m = fmaxf(m, fmaxf(fabsf(__uint_as_float(w4[q] << 16)), fabsf(__uint_as_float(w4[q] & 0xffff0000u))));
+  return m;
 }
 
 }  // namespace
@@ -83,23 +223,139 @@ __device__ bool grid_barrier(uint32_t *bar, DevStatus *st, int *ok_flag) {
 int small_t_grid(int num_sms) { return num_sms; }
 
 size_t small_t_smem_bytes(int T, int H, int k, int I, int Is) {
-  const size_t ng = H / kGroup;
-  const size_t x_bytes = static_cast<size_t>(T) * ng * kXPitch * 4 + static_cast<size_t>(T) * ng * 4;
-  const size_t h_bytes = static_cast<size_t>(T) * (k + 1) * (I > Is ? I : Is) * 4;
-  return x_bytes > h_bytes ? x_bytes : h_bytes;
+  const StLayout L = st_layout(H, I, Is, T, k);
+  if (L.nb < 2 || L.nd < 2) return static_cast<size_t>(1) << 30;  // does not fit: not eligible
+  return L.bytes;
 }
 
-__global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(SmallTArgs a) {
-  extern __shared__ __align__(16) float dyn[];
-  __shared__ SmallTShared sh;
-  const int T = a.T, E = a.E, k = a.k, H = a.H;
-  const int ng = H / kGroup;
-  const int Imax = a.I > a.Is ? a.I : a.Is;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float *xs = dyn;                             // [T][ng][kXPitch]
-  float *xg = dyn + static_cast<size_t>(T) * ng * kXPitch;  // [T][ng] group sums
+bool small_t_fits(int T, int H, int k, int I, int Is, int num_sms) {
+  return T >= 1 && T <= kSmallT && H % 256 == 0 && H / kRowBlock <= small_t_grid(num_sms) &&
+         small_t_smem_bytes(T, H, k, I, Is) <= 220 * 1024;
+}
 
-  // ---- phase 0: routing and staging -------------------------------------------
+__global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs a) {
+  extern __shared__ __align__(1024) uint8_t dyn[];
+  __shared__ SmallTShared sh;
+  const StLayout L = st_layout(a.H, a.I, a.Is, a.T, a.k);
+  const int T = a.T, E = a.E, k = a.k, H = a.H;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, c = lane & 3;  // mma fragment coordinates
+  __half *xs = reinterpret_cast<__half *>(dyn + L.x_off);  // [8][H + kXPad]
+  float *red = reinterpret_cast<float *>(dyn + L.red_off); // [512 threads][8]
+  uint8_t *bring = dyn + L.b_off;
+  uint8_t *dring = dyn + L.d_off;
+  uint64_t *b_full = reinterpret_cast<uint64_t *>(dyn + L.bar_off);
+  uint64_t *d_full = b_full + L.nb;
+  volatile int *abort = &sh.abort;
+  __half *hb = reinterpret_cast<__half *>(a.hbuf);  // [T][k+1][Imax] fp16 scratch, operand order
+  const int Imax = L.Imax;
+  const int nrb_sh = a.Is / kRowBlock;               // the shared expert's row blocks: the first units
+  const int n_dblk = H / kRowBlock;                  // phase-2 output blocks (one per CTA)
+  const int hw = H / 8;                              // packed words per gate/up row
+
+  // ---- phase 0: set-up, routing, token staging, weight requests ------------------
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < L.nb + L.nd; ++s) mbar_init(&b_full[s], 1);
+    sh.abort = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  if (threadIdx.x < kSmallT) sh.xexp[threadIdx.x] = 0;
+  if (threadIdx.x < kMaxExperts / 32) sh.bitmap[threadIdx.x] = 0;
+  for (int i = threadIdx.x; i < kMaxU; i += kSTThreads) {
+    sh.umask[i] = 0;
+#pragma unroll
+    for (int t = 0; t < kSmallT; ++t) sh.uslot[i][t] = -1;
+  }
+  __syncthreads();
+
+  // Phase-1 units are (expert, 16-row block), the shared expert's blocks first;
+  // unit q of this CTA is global unit blockIdx.x + q * gridDim.x and uses ring
+  // stage q % nb. A unit is six bulk copies (gate rows, up rows, their scales
+  // and biases) from lanes 0..5 of warp 0.
+  const int units_per_round = kSTWarps / L.ks;
+  auto issue_b = [&](int q) {  // all lanes of warp 0
+    const int unit = blockIdx.x + q * gridDim.x;
+    int e, rb;
+    if (unit < nrb_sh) {
+      e = E;
+      rb = unit;
+    } else {
+      e = sh.ulist[(unit - nrb_sh) / (a.I / kRowBlock)];
+      rb = (unit - nrb_sh) % (a.I / kRowBlock);
+    }
+    const ExpertPtrs p = expert_ptrs(a, e);
+    uint8_t *st = bring + (q % L.nb) * L.b_stage;
+    const uint32_t pk = kRowBlock * (H / 2), sb = kRowBlock * (H / kGroup) * 2;
+    uint64_t *bar = &b_full[q % L.nb];
+    // the stage's only arrival is this expect-tx, so it cannot complete before
+    // it, whatever order the copies land in
+    if (lane == 0) mbar_arrive_expect_tx(bar, 2 * pk + 4 * sb);
+    if (lane < 2) {
+      const size_t row0 = static_cast<size_t>(lane) * p.Iu + rb * kRowBlock;
+      bulk_g2s(st + lane * pk, p.packed + row0 * hw, pk, bar);
+    } else if (lane < 6) {  // scales / biases, gate then up
+      const int m = (lane - 2) >> 1;
+      const size_t row0 = static_cast<size_t>(m) * p.Iu + rb * kRowBlock;
+      const uint16_t *src = ((lane & 1) ? p.biases : p.scales) + row0 * (H / kGroup);
+      bulk_g2s(st + 2 * pk + (lane - 2) * sb, src, sb, bar);
+    }
+  };
+  // Phase-2 stage u % nd holds expert u's down rows [n0, n0 + 16): three copies,
+  // ten experts per warp-wide step.
+  auto issue_d_range = [&](int u0, int u1) {  // all lanes of warp 0
+    const int n0 = blockIdx.x * kRowBlock;
+    for (int ub = u0; ub < u1; ub += 10) {
+      const int sub = lane / 3, l = lane % 3, u = ub + sub;
+      if (sub < 10 && u < u1) {
+        const ExpertPtrs p = expert_ptrs(a, sh.ulist[u]);
+        uint8_t *st = dring + (u % L.nd) * L.d_stage;
+        const uint32_t pk = kRowBlock * (p.Iu / 2);
+        const uint32_t sb = kRowBlock * (p.Iu / kGroup) * 2;
+        uint64_t *bar = &d_full[u % L.nd];
+        if (l == 0) {
+          mbar_arrive_expect_tx(bar, pk + 2 * sb);
+          bulk_g2s(st, p.packed + static_cast<size_t>(2) * p.Iu * H / 8 + static_cast<size_t>(n0) * (p.Iu / 8), pk,
+                   bar);
+        } else {
+          const size_t g0 = static_cast<size_t>(2) * p.Iu * H / kGroup + static_cast<size_t>(n0) * (p.Iu / kGroup);
+          bulk_g2s(st + kRowBlock * (Imax / 2) + (l - 1) * sb, ((l == 2) ? p.biases : p.scales) + g0, sb, bar);
+        }
+      }
+      __syncwarp();
+    }
+  };
+
+  const bool shared_first = blockIdx.x < nrb_sh;  // unit 0 is a shared-expert block: no routing needed
+  if (warp == 0 && shared_first) issue_b(0);
+
+  // tokens: the upper half of the CTA loads x (kept in registers) and reduces
+  // each token's max |x| while warps 0..T-1 route; a warp's 32 chunks of 8
+  // values belong to one token since H / 8 is a multiple of 32
+  constexpr int kXPer = kSmallT * 2048 / 8 / kSTThreads;  // cached chunks per thread (H <= 2048)
+  const int nxc = T * hw;                                   // 8-value chunks of x
+  const int xt = (threadIdx.x + kSTThreads / 2) % kSTThreads;
+  uint4 xv[kXPer];
+#pragma unroll
+  for (int i = 0; i < kXPer; ++i) {
+    const int idx = xt + i * kSTThreads;
+    xv[i] = make_uint4(0, 0, 0, 0);
+    float m = 0.f;
+    if (idx < nxc) {
+      xv[i] = __ldg(reinterpret_cast<const uint4 *>(a.x) + idx);
+      m = bf16x8_absmax(xv[i]);
+    }
+    m = warp_max(m);
+    const int idx0 = (xt & ~31) + i * kSTThreads;
+    if (lane == 0 && idx0 < nxc && m > 0.f) atomicMax(&sh.xexp[idx0 / hw], __float_as_int(m));
+  }
+  for (int i0 = kXPer * kSTThreads; i0 < nxc; i0 += kSTThreads) {  // H > 2048
+    const int idx = xt + i0, idx0 = (xt & ~31) + i0;
+    float m = 0.f;
+    if (idx < nxc) m = bf16x8_absmax(__ldg(reinterpret_cast<const uint4 *>(a.x) + idx));
+    m = warp_max(m);
+    if (lane == 0 && idx0 < nxc && m > 0.f) atomicMax(&sh.xexp[idx0 / hw], __float_as_int(m));
+  }
   if (warp < T) {
     int id;
     float w;
@@ -107,177 +363,240 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(SmallTArgs a) {
     if (lane < k) {
       sh.ids[warp][lane] = id;
       sh.wt[warp][lane] = w;
+      atomicOr(&sh.bitmap[id >> 5], 1u << (id & 31));
     }
-  }
-  for (int idx = threadIdx.x; idx < T * H / 2; idx += kSTThreads) {
-    const uint32_t v = __ldg(reinterpret_cast<const uint32_t *>(a.x) + idx);
-    const int t = (2 * idx) / H, h = (2 * idx) % H;
-    float *dst = xs + (static_cast<size_t>(t) * ng + h / kGroup) * kXPitch + (h % kGroup);
-    dst[0] = __uint_as_float(v << 16);
-    dst[1] = __uint_as_float(v & 0xffff0000u);
   }
   __syncthreads();
-  for (int idx = threadIdx.x; idx < T * ng; idx += kSTThreads) {
-    const float *src = xs + static_cast<size_t>(idx) * kXPitch;
-    float s = 0.f;
-    for (int i = 0; i < kGroup; ++i) s += src[i];
-    xg[idx] = s;
-  }
+  // distinct experts: the rank of each set bit of the bitmap
   if (warp == 0) {
-    // distinct experts in ascending order, then the shared expert
-    int n = 0;
-    for (int eb = 0; eb < E; eb += 32) {
-      const int e = eb + lane;
-      uint32_t m = 0;
-      int8_t slots[kSmallT];
+    int before = 0;
 #pragma unroll
-      for (int t = 0; t < kSmallT; ++t) slots[t] = -1;
-      if (e < E)
-        for (int t = 0; t < T; ++t)
-          for (int j = 0; j < k; ++j)
-            if (sh.ids[t][j] == e) {
-              m |= 1u << t;
-              slots[t] = static_cast<int8_t>(j);
-            }
-      const unsigned bal = __ballot_sync(0xffffffffu, m != 0);
-      if (m) {
-        const int pos = n + __popc(bal & ((1u << lane) - 1u));
-        sh.ulist[pos] = e;
-        sh.umask[pos] = m;
-#pragma unroll
-        for (int t = 0; t < kSmallT; ++t) sh.uslot[pos][t] = slots[t];
-      }
-      n += __popc(bal);
+    for (int i = 0; i < kMaxExperts / 32; ++i) {
+      const uint32_t wbits = sh.bitmap[i];
+      if ((wbits >> lane) & 1u) sh.ulist[before + __popc(wbits & ((1u << lane) - 1u))] = 32 * i + lane;
+      before += __popc(wbits);
     }
     if (lane == 0) {
-      sh.ulist[n] = E;
-      sh.umask[n] = (1u << T) - 1u;
-      for (int t = 0; t < kSmallT; ++t) sh.uslot[n][t] = static_cast<int8_t>(k);
-      sh.nU = n + 1;
+      sh.ulist[before] = E;
+      sh.umask[before] = (1u << T) - 1u;
+      for (int t = 0; t < T; ++t) sh.uslot[before][t] = static_cast<int8_t>(k);
+      sh.nU = before + 1;
     }
+  } else if (threadIdx.x - 32 < T * k) {  // token/slot pairs: mask and slot of their expert
+    const int f = threadIdx.x - 32, t = f / k, j = f % k, e = sh.ids[t][j];
+    int u = __popc(sh.bitmap[e >> 5] & ((1u << (e & 31)) - 1u));
+    for (int i = 0; i < (e >> 5); ++i) u += __popc(sh.bitmap[i]);
+    atomicOr(&sh.umask[u], 1u << t);
+    sh.uslot[u][t] = static_cast<int8_t>(j);
+  }
+  if (threadIdx.x < kSmallT) {  // per-token power-of-two scale: max |x| in [2, 4) after scaling
+    const float amax = __int_as_float(sh.xexp[threadIdx.x]);
+    int ex = 0;
+    if (amax > 0.f && amax <= 3.0e38f) ex = min(max(ilogbf(amax) - 1, -100), 100);
+    sh.xexp[threadIdx.x] = ex;
   }
   __syncthreads();
   const int nU = sh.nU;
+  const int n_units = nrb_sh + (nU - 1) * (a.I / kRowBlock);
+  const int my_units = blockIdx.x < n_units ? (n_units - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+  const bool has_dblk = blockIdx.x < n_dblk;
+  if (warp == 0) {
+    for (int q = shared_first ? 1 : 0; q < min(my_units, L.nb); ++q) issue_b(q);
+    if (has_dblk) issue_d_range(0, min(nU, L.nd));
+  }
+  // stage the tokens: fp16 scaled by 2^-e in operand order; rows t >= T are zero
+#pragma unroll
+  for (int i = 0; i < kXPer; ++i) {
+    const int idx = xt + i * kSTThreads;
+    if (idx < nxc)
+      *reinterpret_cast<uint4 *>(xs + static_cast<size_t>(idx / hw) * (H + kXPad) + (idx % hw) * 8) =
+          x_scaled_fp16(xv[i], sh.xexp[idx / hw]);
+  }
+  for (int idx = xt + kXPer * kSTThreads; idx < nxc; idx += kSTThreads)
+    *reinterpret_cast<uint4 *>(xs + static_cast<size_t>(idx / hw) * (H + kXPad) + (idx % hw) * 8) =
+        x_scaled_fp16(__ldg(reinterpret_cast<const uint4 *>(a.x) + idx), sh.xexp[idx / hw]);
+  for (int idx = nxc + threadIdx.x; idx < kSmallT * hw; idx += kSTThreads)
+    *reinterpret_cast<uint4 *>(xs + static_cast<size_t>(idx / hw) * (H + kXPad) + (idx % hw) * 8) =
+        make_uint4(0, 0, 0, 0);
+  __syncthreads();
 
-  // ---- phase 1: gate/up ---------------------------------------------------------
-  const int gw = blockIdx.x * kSTWarps + warp, W = gridDim.x * kSTWarps;
-  const int routed_rows = (nU - 1) * a.I;
-  const int total_rows = routed_rows + a.Is;
-  for (int ur = gw; ur < total_rows; ur += W) {
-    int u, i, Iu;
-    const uint32_t *P;
-    const uint16_t *S, *B;
-    if (ur < routed_rows) {
-      u = ur / a.I;
-      i = ur % a.I;
-      Iu = a.I;
-      const size_t e = sh.ulist[u];
-      P = a.w.packed + e * 3 * a.I * H / 8;
-      S = a.w.scales + e * 3 * a.I * H / kGroup;
-      B = a.w.biases + e * 3 * a.I * H / kGroup;
-    } else {
-      u = nU - 1;
-      i = ur - routed_rows;
-      Iu = a.Is;
-      P = a.w.sh_packed;
-      S = a.w.sh_scales;
-      B = a.w.sh_biases;
-    }
-    const uint32_t mask = sh.umask[u];
-    float accg[kSmallT], accu[kSmallT];
+  // ---- phase 1: gate/up ------------------------------------------------------------
+  const int slot = warp / L.ks, kq = warp % L.ks;  // unit slot in a round, K slice of this warp
+  const int rounds = (my_units + units_per_round - 1) / units_per_round;
+  const int ng = H / kGroup;
+  for (int r = 0; r < rounds; ++r) {
+    const int q = r * units_per_round + slot;
+    float accg[4] = {0.f, 0.f, 0.f, 0.f}, accu[4] = {0.f, 0.f, 0.f, 0.f};
+    int u = 0, rb = 0;
+    if (q < my_units) {
+      const int unit = blockIdx.x + q * gridDim.x;
+      if (unit < nrb_sh) {
+        u = nU - 1;
+        rb = unit;
+      } else {
+        u = (unit - nrb_sh) / (a.I / kRowBlock);
+        rb = (unit - nrb_sh) % (a.I / kRowBlock);
+      }
+      const int s = q % L.nb;
+      int ok = 1;
+      if (lane == 0) ok = st_wait(&b_full[s], (q / L.nb) & 1u, abort, a.status, 40) ? 1 : 0;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (ok) {
+        const uint8_t *st = bring + s * L.b_stage;
+        const uint32_t *pg = reinterpret_cast<const uint32_t *>(st);
+        const uint32_t *pu = pg + kRowBlock * hw;
+        const uint16_t *sbp = reinterpret_cast<const uint16_t *>(st + 2 * kRowBlock * (H / 2));
+        const uint16_t *sg = sbp, *bg = sbp + kRowBlock * ng, *su = sbp + 2 * kRowBlock * ng,
+                       *bu = sbp + 3 * kRowBlock * ng;
+        const __half *xrow = xs + static_cast<size_t>(g) * (H + kXPad);
+        for (int wb = kq * L.kw / 8; wb < (kq + 1) * L.kw / 8; wb += 16) {  // blocks of 16 words
+          const int w0 = wb + 4 * c;  // this thread's four words (one scale group)
+          const int grp = w0 / 8;
+          const __half2 sg0 = bf16_to_half2_bcast(sg[g * ng + grp]), bg0 = bf16_to_half2_bcast(bg[g * ng + grp]);
+          const __half2 sg1 = bf16_to_half2_bcast(sg[(g + 8) * ng + grp]),
+                        bg1 = bf16_to_half2_bcast(bg[(g + 8) * ng + grp]);
+          const __half2 su0 = bf16_to_half2_bcast(su[g * ng + grp]), bu0 = bf16_to_half2_bcast(bu[g * ng + grp]);
+          const __half2 su1 = bf16_to_half2_bcast(su[(g + 8) * ng + grp]),
+                        bu1 = bf16_to_half2_bcast(bu[(g + 8) * ng + grp]);
+          const uint4 wg0 = *reinterpret_cast<const uint4 *>(pg + g * hw + w0);
+          const uint4 wg1 = *reinterpret_cast<const uint4 *>(pg + (g + 8) * hw + w0);
+          const uint4 wu0 = *reinterpret_cast<const uint4 *>(pu + g * hw + w0);
+          const uint4 wu1 = *reinterpret_cast<const uint4 *>(pu + (g + 8) * hw + w0);
+          const uint32_t ag0[4] = {wg0.x, wg0.y, wg0.z, wg0.w}, ag1[4] = {wg1.x, wg1.y, wg1.z, wg1.w};
+          const uint32_t au0[4] = {wu0.x, wu0.y, wu0.z, wu0.w}, au1[4] = {wu1.x, wu1.y, wu1.z, wu1.w};
 #pragma unroll
-    for (int t = 0; t < kSmallT; ++t) accg[t] = accu[t] = 0.f;
-    for (int g = lane; g < ng; g += 32) {
-      const uint4 *pg = reinterpret_cast<const uint4 *>(P + static_cast<size_t>(i) * (H / 8) + g * 8);
-      const uint4 *pu = reinterpret_cast<const uint4 *>(P + static_cast<size_t>(Iu + i) * (H / 8) + g * 8);
-      const uint4 g0 = __ldcs(pg), g1 = __ldcs(pg + 1), u0 = __ldcs(pu), u1 = __ldcs(pu + 1);
-      const float sg = bf16_bits_to_float(S[static_cast<size_t>(i) * ng + g]);
-      const float bg = bf16_bits_to_float(B[static_cast<size_t>(i) * ng + g]);
-      const float su = bf16_bits_to_float(S[static_cast<size_t>(Iu + i) * ng + g]);
-      const float bu = bf16_bits_to_float(B[static_cast<size_t>(Iu + i) * ng + g]);
-      const uint32_t gw8[8] = {g0.x, g0.y, g0.z, g0.w, g1.x, g1.y, g1.z, g1.w};
-      const uint32_t uw8[8] = {u0.x, u0.y, u0.z, u0.w, u1.x, u1.y, u1.z, u1.w};
-#pragma unroll
-      for (int t = 0; t < kSmallT; ++t) {
-        if (t >= T || !((mask >> t) & 1u)) continue;
-        const float *xr = xs + (static_cast<size_t>(t) * ng + g) * kXPitch;
-        float dg = 0.f, du = 0.f;
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          float xv[8];
-          *reinterpret_cast<float4 *>(&xv[0]) = *reinterpret_cast<const float4 *>(xr + 8 * q);
-          *reinterpret_cast<float4 *>(&xv[4]) = *reinterpret_cast<const float4 *>(xr + 8 * q + 4);
-          dg += dot8(gw8[q], xv);
-          du += dot8(uw8[q], xv);
+          for (int p = 0; p < 4; ++p) {
+            const uint4 xb = *reinterpret_cast<const uint4 *>(xrow + (w0 + p) * 8);
+            const uint4 g0 = dequant_word(ag0[p], sg0, bg0), g1 = dequant_word(ag1[p], sg1, bg1);
+            const uint4 u0 = dequant_word(au0[p], su0, bu0), u1 = dequant_word(au1[p], su1, bu1);
+            mma16816(accg, g0.x, g1.x, g0.y, g1.y, xb.x, xb.y);
+            mma16816(accg, g0.z, g1.z, g0.w, g1.w, xb.z, xb.w);
+            mma16816(accu, u0.x, u1.x, u0.y, u1.y, xb.x, xb.y);
+            mma16816(accu, u0.z, u1.z, u0.w, u1.w, xb.z, xb.w);
+          }
         }
-        const float xsum = xg[t * ng + g];
-        accg[t] += sg * dg + bg * xsum;
-        accu[t] += su * du + bu * xsum;
       }
     }
+    // partial sums of the K slices, reduced in slice order by the unit's first warp
+    float *rp = red + static_cast<size_t>(threadIdx.x) * 8;
 #pragma unroll
-    for (int t = 0; t < kSmallT; ++t) {
-      if (t >= T || !((mask >> t) & 1u)) continue;
-      const float G = warp_sum(accg[t]), U = warp_sum(accu[t]);
-      if (lane == 0) {
-        const int j = sh.uslot[u][t];
-        a.hbuf[(static_cast<size_t>(t) * (k + 1) + j) * Imax + i] = G / (1.0f + __expf(-G)) * U;
+    for (int i = 0; i < 4; ++i) {
+      rp[i] = accg[i];
+      rp[4 + i] = accu[i];
+    }
+    __syncthreads();
+    if (q < my_units && kq == 0) {
+      float G[4] = {0.f, 0.f, 0.f, 0.f}, U[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int zz = 0; zz < L.ks; ++zz) {
+        const float *zp = red + static_cast<size_t>((warp + zz) * 32 + lane) * 8;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          G[i] += zp[i];
+          U[i] += zp[4 + i];
+        }
+      }
+      // C fragment: rows g (i = 0, 1) and g + 8 (i = 2, 3), token columns 2c, 2c + 1
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int t = 2 * c + (i & 1);
+        const int row = rb * kRowBlock + g + (i >> 1) * 8;
+        if (t < T && ((sh.umask[u] >> t) & 1u)) {
+          const int j = sh.uslot[u][t];
+          const float hv = swiglu_scaled(G[i], U[i], sh.xexp[t]);
+          hb[(static_cast<size_t>(t) * (k + 1) + j) * Imax + (row & ~7) + kperm_dst(row & 7)] = __float2half_rn(hv);
+        }
+      }
+    }
+    __syncthreads();
+    // the stages this round used are free: refill them with the units nb ahead
+    if (warp == 0)
+      for (int zz = 0; zz < units_per_round; ++zz) {
+        const int qn = r * units_per_round + zz + L.nb;
+        if (qn < my_units) issue_b(qn);
+      }
+  }
+
+  // ---- grid barrier ------------------------------------------------------------------
+  if (!grid_barrier(a.barrier, a.status, &sh.ok)) return;
+
+  // ---- phase 2: down + combine -------------------------------------------------------
+  if (!has_dblk) return;
+  // copy the tokens' h (all slots) into the phase-1 ring, which is free now
+  __half *hs = reinterpret_cast<__half *>(bring);
+  const int hchunks = T * (k + 1) * Imax / 8;
+  for (int i = threadIdx.x; i < hchunks; i += kSTThreads)
+    reinterpret_cast<uint4 *>(hs)[i] = __ldcg(reinterpret_cast<const uint4 *>(hb) + i);
+  __syncthreads();
+  const int n0 = blockIdx.x * kRowBlock;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};  // rows g, g+8; tokens 2c, 2c+1 (this warp's experts, ascending)
+  bool ok2 = true;
+  for (int base = 0; base < nU; base += L.nd) {
+    const uint32_t par = (base / L.nd) & 1u;
+    if (base > 0) {  // next pass: the ring's stages are free once every warp is done
+      __syncthreads();
+      if (warp == 0) issue_d_range(base, min(nU, base + L.nd));
+    }
+    for (int u = base + warp; u < min(nU, base + L.nd); u += kSTWarps) {
+      const int s = u % L.nd;
+      int ok = ok2 ? 1 : 0;
+      if (lane == 0 && ok) ok = st_wait(&d_full[s], par, abort, a.status, 41) ? 1 : 0;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      ok2 = ok != 0;
+      if (!ok2) continue;
+      const int Iu = sh.ulist[u] == E ? a.Is : a.I;
+      const int iw = Iu / 8;  // packed words per down row
+      const uint8_t *st = dring + s * L.d_stage;
+      const uint32_t *pd = reinterpret_cast<const uint32_t *>(st);
+      const int ngd = Iu / kGroup;
+      const uint16_t *sd = reinterpret_cast<const uint16_t *>(st + kRowBlock * (Imax / 2));
+      const uint16_t *bd = sd + kRowBlock * ngd;
+      // B fragments: token g's h for this expert (zeros if g is not routed to it)
+      const int jg = (g < T) ? sh.uslot[u][g] : -1;
+      const __half *hrow = hs + (static_cast<size_t>(g) * (k + 1) + (jg < 0 ? 0 : jg)) * Imax;
+      float y[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int wb = 0; wb < iw; wb += 16) {
+        const int w0 = wb + 4 * c;
+        const int grp = w0 / 8;
+        const __half2 s0 = bf16_to_half2_bcast(sd[g * ngd + grp]), b0 = bf16_to_half2_bcast(bd[g * ngd + grp]);
+        const __half2 s1 = bf16_to_half2_bcast(sd[(g + 8) * ngd + grp]),
+                      b1 = bf16_to_half2_bcast(bd[(g + 8) * ngd + grp]);
+        const uint4 wd0 = *reinterpret_cast<const uint4 *>(pd + g * iw + w0);
+        const uint4 wd1 = *reinterpret_cast<const uint4 *>(pd + (g + 8) * iw + w0);
+        const uint32_t ad0[4] = {wd0.x, wd0.y, wd0.z, wd0.w}, ad1[4] = {wd1.x, wd1.y, wd1.z, wd1.w};
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+          uint4 hbv = make_uint4(0, 0, 0, 0);
+          if (jg >= 0) hbv = *reinterpret_cast<const uint4 *>(hrow + (w0 + p) * 8);
+          const uint4 d0 = dequant_word(ad0[p], s0, b0), d1 = dequant_word(ad1[p], s1, b1);
+          mma16816(y, d0.x, d1.x, d0.y, d1.y, hbv.x, hbv.y);
+          mma16816(y, d0.z, d1.z, d0.w, d1.w, hbv.z, hbv.w);
+        }
+      }
+      // weight each token's column by its routing weight (1 for the shared expert) and 2^(2e)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int t = 2 * c + (i & 1);
+        if (t < T && ((sh.umask[u] >> t) & 1u)) {
+          const int j = sh.uslot[u][t];
+          const float wgt = (j == k) ? 1.0f : sh.wt[t][j];
+          acc[i] += wgt * ldexpf(y[i], 2 * sh.xexp[t]);
+        }
       }
     }
   }
-
-  // ---- grid barrier ---------------------------------------------------------------
-  if (!grid_barrier(a.barrier, a.status, &sh.ok)) return;
-
-  // ---- phase 2: down + combine -----------------------------------------------------
-  float *hp = dyn;  // [T][k+1][Imax], reuses the x staging area
-  const int npair = T * (k + 1);
-  for (int idx = threadIdx.x; idx < npair * Imax / 4; idx += kSTThreads)
-    reinterpret_cast<float4 *>(hp)[idx] = __ldcg(reinterpret_cast<const float4 *>(a.hbuf) + idx);
+  float *rp = red + static_cast<size_t>(threadIdx.x) * 8;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) rp[i] = acc[i];
   __syncthreads();
-  for (int n = gw; n < H; n += W) {
-    for (int t = 0; t < T; ++t) {
-      float acc = 0.f;
-      for (int j = 0; j <= k; ++j) {
-        const bool shared = j == k;
-        const int Iu = shared ? a.Is : a.I;
-        const uint32_t *P;
-        const uint16_t *S, *B;
-        if (shared) {
-          P = a.w.sh_packed;
-          S = a.w.sh_scales;
-          B = a.w.sh_biases;
-        } else {
-          const size_t e = sh.ids[t][j];
-          P = a.w.packed + e * 3 * a.I * H / 8;
-          S = a.w.scales + e * 3 * a.I * H / kGroup;
-          B = a.w.biases + e * 3 * a.I * H / kGroup;
-        }
-        P += static_cast<size_t>(2) * Iu * H / 8 + static_cast<size_t>(n) * (Iu / 8);
-        S += static_cast<size_t>(2) * Iu * H / kGroup + static_cast<size_t>(n) * (Iu / kGroup);
-        B += static_cast<size_t>(2) * Iu * H / kGroup + static_cast<size_t>(n) * (Iu / kGroup);
-        const float *hv = hp + (static_cast<size_t>(t) * (k + 1) + j) * Imax;
-        float part = 0.f;
-        for (int w2 = lane; w2 < Iu / 16; w2 += 32) {
-          const uint2 wd = __ldcs(reinterpret_cast<const uint2 *>(P) + w2);
-          const int g = w2 / 4;
-          const float s = bf16_bits_to_float(S[g]), b = bf16_bits_to_float(B[g]);
-          const float *hr = hv + 16 * w2;
-          float hx[16];
+  // warps' contributions summed in warp order, one rounding; 16 rows x T tokens
+  if (warp == 0) {
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
-            *reinterpret_cast<float4 *>(&hx[4 * q]) = *reinterpret_cast<const float4 *>(hr + 4 * q);
-          const float d = dot8(wd.x, hx) + dot8(wd.y, hx + 8);
-          float hs = 0.f;
-#pragma unroll
-          for (int q = 0; q < 16; ++q) hs += hx[q];
-          part += s * d + b * hs;
-        }
-        const float y = warp_sum(part);
-        acc += (shared ? 1.0f : sh.wt[t][j]) * y;
-      }
-      if (lane == 0) {
-        float o = acc;
+    for (int i = 0; i < 4; ++i) {
+      const int t = 2 * c + (i & 1);
+      const int n = n0 + g + (i >> 1) * 8;
+      if (t < T) {
+        float o = 0.f;
+        for (int zz = 0; zz < kSTWarps; ++zz) o += red[static_cast<size_t>(zz * 32 + lane) * 8 + i];
         if (a.residual) o += bf16_bits_to_float(a.residual[static_cast<size_t>(t) * H + n]);
         a.out[static_cast<size_t>(t) * H + n] = float_to_bf16_bits(o);
       }
@@ -286,7 +605,8 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(SmallTArgs a) {
 }
 
 cudaError_t launch_small_t(const SmallTArgs &a, int num_sms, cudaStream_t s) {
-  const size_t smem = small_t_smem_bytes(a.T, a.H, a.k, a.I, a.Is);
+  const StLayout L = st_layout(a.H, a.I, a.Is, a.T, a.k);
+  const size_t smem = L.bytes;
   cudaError_t err = cudaFuncSetAttribute(small_t_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
   if (err != cudaSuccess) return err;

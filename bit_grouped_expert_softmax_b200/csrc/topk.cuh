@@ -34,9 +34,21 @@ __device__ __forceinline__ int warp_incl_scan(int v) {
   return v;
 }
 
+// Order-preserving unsigned key of a float (larger float -> larger key).
+__device__ __forceinline__ uint32_t float_key(float f) {
+  const uint32_t u = __float_as_uint(f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key_float(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
 // Top-k of one token by one warp. Lane l holds experts l, l+32, ... (E <= 256).
-// Writes the token's k ids (largest logit first) and weights to lanes 0..k-1's
-// out_id / out_w. Every lane returns the same psum.
+// Each round takes the largest remaining float32 logit (two warp reductions:
+// the maximum key, then the lowest expert id holding it), so equal logits go
+// to the lower id. Lanes 0..k-1 return the chosen ids (largest logit first)
+// in out_id and their weights in out_w: the softmax over all E experts (fp32,
+// max-subtracted) restricted to the chosen k and renormalised to sum to one.
 __device__ __forceinline__ void warp_topk(const float *__restrict__ row, int E, int k, int lane,
                                           int &out_id, float &out_w) {
   float v[8];
@@ -45,50 +57,41 @@ __device__ __forceinline__ void warp_topk(const float *__restrict__ row, int E, 
     const int e = lane + 32 * i;
     v[i] = (e < E) ? __ldg(row + e) : -INFINITY;
   }
-  // softmax over all E experts (fp32, max-subtracted)
-  float m = v[0];
-#pragma unroll
-  for (int i = 1; i < 8; ++i) m = fmaxf(m, v[i]);
-  m = warp_max(m);
-  float z = 0.f;
-#pragma unroll
-  for (int i = 0; i < 8; ++i)
-    if (lane + 32 * i < E) z += expf(v[i] - m);
-  z = warp_sum(z);
-
-  uint32_t taken = 0;
-  float psum = 0.f, my_p = 0.f;
+  uint32_t taken = 0, my_key = 0;
   int my_id = 0;
+  float m = 0.f, z = 0.f;
   for (int j = 0; j < k; ++j) {
-    float bv = -INFINITY;
+    uint32_t bk = 0;  // 0: no candidate in this lane (every float key is > 0)
     int bi = 0x7fffffff;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int e = lane + 32 * i;
-      if (e < E && !(taken >> i & 1u) && better(v[i], e, bv, bi)) {
-        bv = v[i];
+      const uint32_t kk = float_key(v[i]);
+      if (e < E && !(taken >> i & 1u) && kk > bk) {  // ascending e: ties keep the lower id
+        bk = kk;
         bi = e;
       }
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-      if (better(ov, oi, bv, bi)) {
-        bv = ov;
-        bi = oi;
-      }
-    }
-    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
-    const float p = expf(bv - m) / z;  // softmax probability of the chosen expert
-    psum += p;
+    const uint32_t mk = __reduce_max_sync(0xffffffffu, bk);
+    const int win = static_cast<int>(__reduce_min_sync(0xffffffffu, bk == mk ? static_cast<uint32_t>(bi) : 0xffffffffu));
+    if ((win & 31) == lane) taken |= 1u << (win >> 5);
     if (lane == j) {
-      my_id = bi;
-      my_p = p;
+      my_id = win;
+      my_key = mk;
+    }
+    if (j == 0) {  // the first pick is the maximum: softmax denominator over all E
+      m = key_float(mk);
+      float zz = 0.f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        if (lane + 32 * i < E) zz += expf(v[i] - m);
+      z = warp_sum(zz);
     }
   }
+  const float p = (lane < k) ? expf(key_float(my_key) - m) / z : 0.f;  // softmax probability
+  const float psum = warp_sum(p);
   out_id = my_id;
-  out_w = my_p / psum;  // renormalise the k chosen probabilities to sum to one
+  out_w = p / psum;  // renormalise the k chosen probabilities to sum to one
 }
 
 }  // namespace moe
