@@ -141,7 +141,62 @@ def run_gpu(args, rank, world, local_rank):
     peaks, peaks_kind = load_peaks()
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
 
+    def measure_stack(steps, warmup):
+        """One step = the whole stack of layers over one T-token chunk."""
+        wl = synth.WORKLOADS["stack"]
+        layers, logits, rfs = [], [], []
+        for l in range(wl.layers):
+            inp = synth.make_stack_layer(wl, l)
+            layers.append(api.DeviceLayer.from_inputs(inp, dev))
+            logits.append(inp.logits)
+            rfs.append(roofline_numbers(inp, peaks))
+        rf = dict(rfs[0])
+        rf["weight_bytes"] = sum(r["weight_bytes"] for r in rfs)
+        rf["flops"] = sum(r["flops"] for r in rfs)
+        rf["touched"] = rfs[0]["touched"]
+        rf["t_hbm"] = rf["weight_bytes"] / (peaks["hbm_gbs"] * 1e9)
+        rf["t_tc"] = rf["flops"] / (peaks["bf16_tflops"] * 1e12)
+        rf["bound"] = "hbm" if rf["t_hbm"] >= rf["t_tc"] else "tensor"
+        x0 = torch.from_numpy(synth.make_stack_x(wl).view(np.int16)).to(dev)
+        x = x0.clone()
+        dlog = torch.from_numpy(np.stack(logits)).to(dev)
+        plan = api.Plan(wl.T, wl.H, wl.E, wl.k, wl.I, wl.Is)
+        stream = torch.cuda.Stream(dev)
+        torch.cuda.set_stream(stream)
+
+        def step(i):
+            x.copy_(x0)
+            api.moe_stack_forward(plan.handle, wl.layers, wl.T, x, dlog, layers, stream)
+
+        for i in range(warmup):
+            step(i)
+        plan.status_sync(stream)
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        with ClockSampler(local_rank) as clk:
+            e0.record(stream)
+            for i in range(steps):
+                step(i)
+            e1.record(stream)
+            torch.cuda.synchronize(dev)
+        ms_step = e0.elapsed_time(e1) / steps
+        api.moe_profile_enable(plan.handle, 8 * wl.layers * 2)
+        for i in range(2):
+            step(i)
+        prof = api.moe_profile_read(plan.handle, stream)
+        api.moe_profile_enable(plan.handle, 0)
+        plan.status_sync(stream)
+        res = dict(workload="stack", T=wl.T, ms_per_step=ms_step, tokens_s=wl.T * world / (ms_step * 1e-3), rf=rf,
+                   achieved_gbs=rf["weight_bytes"] / (ms_step * 1e-3) / 1e9,
+                   achieved_tflops=rf["flops"] / (ms_step * 1e-3) / 1e12, n_rep=1, graph=False,
+                   timed_steps=steps, clocks=clk.summary(), e2e_tokens_s=None, h2d=0, d2h=0,
+                   launches=7 * wl.layers * steps, inp=None, prof=prof, layers=wl.layers)
+        plan.close()
+        return res
+
     def measure(name, steps, warmup):
+        if name == "stack":
+            return measure_stack(steps, warmup)
         inp = synth.make_workload(name)
         rf = roofline_numbers(inp, peaks)
         base = api.DeviceLayer.from_inputs(inp, dev)
@@ -268,7 +323,8 @@ def roofline_obj(r, peaks, peaks_kind):
     ms, n = prof[name]
     avg_s = ms * 1e-3 / max(n, 1)
     fb, ff = KERNEL_SHARE.get(name, (0.0, 0.0))
-    kbytes, kflops = rf["weight_bytes"] * fb, rf["flops"] * ff
+    per_launch = 1.0 / r.get("layers", 1)  # the stack's totals cover every layer; a launch is one layer
+    kbytes, kflops = rf["weight_bytes"] * fb * per_launch, rf["flops"] * ff * per_launch
     t_hbm = kbytes / (peaks["hbm_gbs"] * 1e9)
     t_tc = kflops / (peaks["bf16_tflops"] * 1e12)
     if t_hbm >= t_tc:
@@ -286,7 +342,7 @@ def summarize_extra(r, peaks, peaks_kind):
             "effective_tflops": round(r["achieved_tflops"], 2), "achieved_weight_gbs": round(r["achieved_gbs"], 1),
             "roofline": roofline_obj(r, peaks, peaks_kind), "kernels": kernel_table(r), "graph": r["graph"],
             "clocks": r["clocks"],
-            "e2e_tokens_s": round(r["e2e_tokens_s"], 1)}
+            "e2e_tokens_s": None if r["e2e_tokens_s"] is None else round(r["e2e_tokens_s"], 1)}
 
 
 def cpu_baseline(name, budget_s=15.0):
@@ -316,7 +372,7 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
-    ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "zipf", "tiny"])
+    ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "zipf", "tiny", "stack"])
     ap.add_argument("--no-extra", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--replicas", type=int, default=0,
@@ -383,7 +439,7 @@ def main():
                 "kernels": kernel_table(r),
                 "effective_tflops": round(r["achieved_tflops"], 3),
                 "cpu_baseline": cpu,
-                "e2e": {"value": round(r["e2e_tokens_s"], 1), "unit": "tokens/s",
+                "e2e": {"value": None if r["e2e_tokens_s"] is None else round(r["e2e_tokens_s"], 1), "unit": "tokens/s",
                         "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]},
                 "gpu_launches": r["launches"], "clocks": r["clocks"], "extra": extra}
         print(json.dumps(line))
