@@ -40,6 +40,21 @@ METRIC = "MoE-layer tokens/s"
 PEAKS_FALLBACK = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
+def reduce_max(value: float, world: int, device=None) -> float:
+    """Maximum of a per-rank value over all ranks (device time: the slowest rank)."""
+    if world <= 1:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tokens_s(tokens_per_rank: int, world: int, ms_per_step: float) -> float:
+    """Tokens all ranks processed per second, timed by the slowest rank."""
+    return tokens_per_rank * world / (ms_per_step * 1e-3)
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -179,14 +194,14 @@ def run_gpu(args, rank, world, local_rank):
                 step(i)
             e1.record(stream)
             torch.cuda.synchronize(dev)
-        ms_step = e0.elapsed_time(e1) / steps
+        ms_step = reduce_max(e0.elapsed_time(e1), world, dev) / steps
         api.moe_profile_enable(plan.handle, 8 * wl.layers * 2)
         for i in range(2):
             step(i)
         prof = api.moe_profile_read(plan.handle, stream)
         api.moe_profile_enable(plan.handle, 0)
         plan.status_sync(stream)
-        res = dict(workload="stack", T=wl.T, ms_per_step=ms_step, tokens_s=wl.T * world / (ms_step * 1e-3), rf=rf,
+        res = dict(workload="stack", T=wl.T, ms_per_step=ms_step, tokens_s=whole_job_tokens_s(wl.T, world, ms_step), rf=rf,
                    achieved_gbs=rf["weight_bytes"] / (ms_step * 1e-3) / 1e9,
                    achieved_tflops=rf["flops"] / (ms_step * 1e-3) / 1e12, n_rep=1, graph=False,
                    timed_steps=steps, clocks=clk.summary(), e2e_tokens_s=None, h2d=0, d2h=0,
@@ -254,12 +269,9 @@ def run_gpu(args, rank, world, local_rank):
             torch.cuda.synchronize(dev)
         ms = e0.elapsed_time(e1)
         plan.status_sync(stream)
-        if world > 1:
-            t = torch.tensor([ms], device=dev)
-            torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-            ms = float(t.item())
+        ms = reduce_max(ms, world, dev)
         ms_step = ms / timed_steps
-        tokens_s = inp.T * world / (ms_step * 1e-3)
+        tokens_s = whole_job_tokens_s(inp.T, world, ms_step)
         # end to end through the host-buffer entry point (pinned host memory)
         xh = torch.from_numpy(inp.x.view(np.int16)).pin_memory()
         lh = torch.from_numpy(inp.logits).pin_memory()
@@ -307,6 +319,24 @@ def run_gpu(args, rank, world, local_rank):
 KERNEL_SHARE = {"small_t": (1.0, 1.0), "gate_up": (2 / 3, 2 / 3), "down": (1 / 3, 1 / 3)}
 
 
+def measured_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from the committed ncu capture of this kernel and
+    workload, or None if there is none or the kernel's sources changed since."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        rec = json.load(f).get(kernel)
+    if not rec or rec.get("workload") != workload:
+        return None
+    h = hashlib.sha256()
+    for src in rec["sources"]:
+        with open(os.path.join(ROOT, src), "rb") as f:
+            h.update(f.read())
+    return rec["dram_bytes_per_launch"] if h.hexdigest()[:16] == rec["sha"] else None
+
+
 def kernel_table(r):
     prof = r["prof"]
     tot = sum(v[0] for v in prof.values()) or 1.0
@@ -332,7 +362,8 @@ def roofline_obj(r, peaks, peaks_kind):
     else:
         a, p, unit, bound = kflops / avg_s / 1e12, peaks["bf16_tflops"], "TFLOP/s", "tensor"
     return {"bound": bound, "achieved": round(a, 2), "peak": p, "unit": unit, "frac": round(a / p, 4),
-            "traffic": None, "peak_source": peaks_kind, "kernel": name, "kernel_avg_us": round(avg_s * 1e6, 3),
+            "traffic": measured_traffic(name, r["workload"]), "traffic_unit": "bytes per launch (ncu)",
+            "peak_source": peaks_kind, "kernel": name, "kernel_avg_us": round(avg_s * 1e6, 3),
             "algorithmic_per_launch": {"weight_bytes": int(kbytes), "flops": kflops,
                                        "touched_experts_incl_shared": rf["touched"]}}
 
