@@ -42,21 +42,21 @@ constexpr int kMmaWarp = 2;            // MMA issuer
 constexpr int kEpiWarp0 = 3;           // warps 3..6: epilogue
 constexpr int kDqWarp0 = 7;            // warps 7..14: dequantisation
 constexpr int kDqWarps = 8;
-constexpr int kStageK = 2;             // 64-wide K-blocks per A/B pipeline stage
+constexpr int kStageK = 2;             // 64-wide K-blocks per activation stage
 constexpr int kBStages = 3;            // activation ring (smem)
-constexpr int kAStages = 2;            // dequantised weights (TMEM)
 constexpr int kBRows = 32;             // TMA box height of activation rows
 constexpr int kBAtomBytes = kTileN * 128;          // 128 rows x 64 fp16
 constexpr int kBStageBytes = kStageK * kBAtomBytes;
 constexpr int kSuperK = 4;             // K-blocks per packed stage (128-byte rows of words)
 constexpr int kPkTileBytes = kTileM * 128;         // 128 rows x 32 words
 constexpr int kAccCols = kTileN;       // fp32 accumulator columns per matrix
-constexpr int kAColsPerMat = kStageK * 32;         // TMEM columns of one matrix in one A stage
+constexpr int kAColsPerMat = 32;       // TMEM columns of one matrix in one A stage (one 64-wide K-block)
 
 template <int NMAT>
 struct Cfg {
   static constexpr int kPkStages = NMAT == 2 ? 3 : 4;
   static constexpr int kAccStages = NMAT == 2 ? 1 : 2;  // TMEM: accumulators then A stages
+  static constexpr int kAStages = NMAT == 2 ? 4 : 8;    // dequantised weights (TMEM), one K-block each
   static constexpr int kACol0 = kAccStages * NMAT * kAccCols;
   static constexpr int kTmemCols = 512;
   static_assert(kACol0 + kAStages * NMAT * kAColsPerMat <= kTmemCols, "TMEM budget");
@@ -140,8 +140,8 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
   uint64_t *b_full = pk_empty + C::kPkStages;
   uint64_t *b_empty = b_full + kBStages;
   uint64_t *a_full = b_empty + kBStages;
-  uint64_t *a_empty = a_full + kAStages;
-  uint64_t *acc_full = a_empty + kAStages;
+  uint64_t *a_empty = a_full + C::kAStages;
+  uint64_t *acc_full = a_empty + C::kAStages;
   uint64_t *acc_empty = acc_full + C::kAccStages;
   uint64_t *mma_done = acc_empty + C::kAccStages;
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + C::kOffMisc);
@@ -159,7 +159,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
       mbar_init(&b_full[s], 1);
       mbar_init(&b_empty[s], 1);
     }
-    for (int s = 0; s < kAStages; ++s) {
+    for (int s = 0; s < C::kAStages; ++s) {
       mbar_init(&a_full[s], kDqWarps);
       mbar_init(&a_empty[s], 1);
     }
@@ -286,35 +286,40 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
       const uint32_t idesc = idesc_f16_f32(kTileM, n16);
       const uint32_t d0 = tmem_base + st * NMAT * kAccCols;
       for (int ks = 0; ks < K / (kTileK * kStageK); ++ks) {
-        if (!warp_wait(&a_full[sa], pha, abort, a.status, 111) || !warp_wait(&b_full[sb], phb, abort, a.status, 112)) {
+        if (!warp_wait(&b_full[sb], phb, abort, a.status, 112)) {
           ok = false;
           break;
         }
-        tc_fence_after();
-        if (elect_one()) {
-          const uint32_t b_addr = smem_u32(sB + sb * kBStageBytes);
-          const uint32_t a_col = tmem_base + C::kACol0 + sa * NMAT * kAColsPerMat;
-#pragma unroll
-          for (int kh = 0; kh < kStageK; ++kh)
+        const uint32_t b_addr = smem_u32(sB + sb * kBStageBytes);
+        for (int kh = 0; kh < kStageK; ++kh) {
+          if (!warp_wait(&a_full[sa], pha, abort, a.status, 111)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (elect_one()) {
+            const uint32_t a_col = tmem_base + C::kACol0 + sa * NMAT * kAColsPerMat;
 #pragma unroll
             for (int kk = 0; kk < kTileK / 16; ++kk) {
               const uint64_t bdesc = smem_desc_sw128(b_addr + kh * kBAtomBytes + kk * 32);
 #pragma unroll
               for (int m = 0; m < NMAT; ++m)
-                tc_mma_f16_ts(d0 + m * kAccCols, a_col + m * kAColsPerMat + kh * 32 + kk * 8, bdesc, idesc,
+                tc_mma_f16_ts(d0 + m * kAccCols, a_col + m * kAColsPerMat + kk * 8, bdesc, idesc,
                               (ks | kh | kk) != 0 ? 1u : 0u);
             }
-          tc_commit(&b_empty[sb]);
-          tc_commit(&a_empty[sa]);
+            tc_commit(&a_empty[sa]);
+            if (kh == kStageK - 1) tc_commit(&b_empty[sb]);
+          }
+          __syncwarp();
+          if (++sa == C::kAStages) {
+            sa = 0;
+            pha ^= 1u;
+          }
         }
-        __syncwarp();
+        if (!ok) break;
         if (++sb == kBStages) {
           sb = 0;
           phb ^= 1u;
-        }
-        if (++sa == kAStages) {
-          sa = 0;
-          pha ^= 1u;
         }
       }
       if (ok && elect_one()) tc_commit(&acc_full[st]);
@@ -453,80 +458,75 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
       }
       const int nkb = K / kTileK;  // one scale/bias group per K-block
       uint16_t s_next = __ldg(S), b_next = __ldg(B);
-      for (int kb0 = 0; kb0 < nkb; kb0 += kStageK) {
+      for (int kb = 0; kb < nkb; ++kb) {
         if (!warp_wait(&a_empty[sa], pha ^ 1u, abort, a.status, 131)) {
           ok = false;
           break;
         }
         const uint32_t ta =
             tmem_base + (static_cast<uint32_t>(q * 32) << 16) + C::kACol0 + sa * NMAT * kAColsPerMat + m * kAColsPerMat;
-#pragma unroll
-        for (int kh = 0; kh < kStageK; ++kh) {
-          const int kb = kb0 + kh;
-          const __half2 s2 = bf16_to_half2_bcast(s_next), b2 = bf16_to_half2_bcast(b_next);
-          if (kb + 1 < nkb) {
-            s_next = __ldg(S + kb + 1);
-            b_next = __ldg(B + kb + 1);
-          }
-          const int j = kb % kSuperK;
-          if (j == 0 && !warp_wait(&pk_full[sp], php, abort, a.status, 130)) {
-            ok = false;
-            break;
-          }
-          // row r of the packed stage: 128 bytes = 4 K-blocks of 8 words, in
-          // 16-byte chunks placed at chunk ^ (r & 7) by the TMA's 128-byte swizzle
-          const uint8_t *prow = sPk + (sp * NMAT + m) * kPkTileBytes + r * 128;
-          if (gate_up) {
-            const uint4 v0 = *reinterpret_cast<const uint4 *>(prow + (((2 * j) ^ (r & 7)) << 4));
-            const uint4 v1 = *reinterpret_cast<const uint4 *>(prow + (((2 * j + 1) ^ (r & 7)) << 4));
-            if (j == kSuperK - 1 || kb == nkb - 1) {  // words in registers: release the packed stage
-              __syncwarp();
-              if (lane == 0) mbar_arrive(&pk_empty[sp]);
-              if (++sp == C::kPkStages) {
-                sp = 0;
-                php ^= 1u;
-              }
-            }
-            const uint32_t wv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-            uint32_t d[32];
-#pragma unroll
-            for (int cw = 0; cw < 8; ++cw) {
-              const uint4 v = dequant_word(wv[cw], s2, b2);
-              d[4 * cw + 0] = v.x;
-              d[4 * cw + 1] = v.y;
-              d[4 * cw + 2] = v.z;
-              d[4 * cw + 3] = v.w;
-            }
-            tmem_st_32x32b_x32(ta + kh * 32, d);
-          } else {
-            const uint4 v0 = *reinterpret_cast<const uint4 *>(prow + (((2 * j + half) ^ (r & 7)) << 4));
-            if (j == kSuperK - 1 || kb == nkb - 1) {
-              __syncwarp();
-              if (lane == 0) mbar_arrive(&pk_empty[sp]);
-              if (++sp == C::kPkStages) {
-                sp = 0;
-                php ^= 1u;
-              }
-            }
-            const uint32_t wv[4] = {v0.x, v0.y, v0.z, v0.w};
-            uint32_t d[16];
-#pragma unroll
-            for (int cw = 0; cw < 4; ++cw) {
-              const uint4 v = dequant_word(wv[cw], s2, b2);
-              d[4 * cw + 0] = v.x;
-              d[4 * cw + 1] = v.y;
-              d[4 * cw + 2] = v.z;
-              d[4 * cw + 3] = v.w;
-            }
-            tmem_st_32x32b_x16(ta + kh * 32 + 16 * half, d);
-          }
+        const __half2 s2 = bf16_to_half2_bcast(s_next), b2 = bf16_to_half2_bcast(b_next);
+        if (kb + 1 < nkb) {
+          s_next = __ldg(S + kb + 1);
+          b_next = __ldg(B + kb + 1);
         }
-        if (!ok) break;
+        const int j = kb % kSuperK;
+        if (j == 0 && !warp_wait(&pk_full[sp], php, abort, a.status, 130)) {
+          ok = false;
+          break;
+        }
+        // row r of the packed stage: 128 bytes = 4 K-blocks of 8 words, in
+        // 16-byte chunks placed at chunk ^ (r & 7) by the TMA's 128-byte swizzle
+        const uint8_t *prow = sPk + (sp * NMAT + m) * kPkTileBytes + r * 128;
+        if (gate_up) {
+          const uint4 v0 = *reinterpret_cast<const uint4 *>(prow + (((2 * j) ^ (r & 7)) << 4));
+          const uint4 v1 = *reinterpret_cast<const uint4 *>(prow + (((2 * j + 1) ^ (r & 7)) << 4));
+          if (j == kSuperK - 1 || kb == nkb - 1) {  // words in registers: release the packed stage
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&pk_empty[sp]);
+            if (++sp == C::kPkStages) {
+              sp = 0;
+              php ^= 1u;
+            }
+          }
+          const uint32_t wv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+          uint32_t d[32];
+#pragma unroll
+          for (int cw = 0; cw < 8; ++cw) {
+            const uint4 v = dequant_word(wv[cw], s2, b2);
+            d[4 * cw + 0] = v.x;
+            d[4 * cw + 1] = v.y;
+            d[4 * cw + 2] = v.z;
+            d[4 * cw + 3] = v.w;
+          }
+          tmem_st_32x32b_x32(ta, d);
+        } else {
+          const uint4 v0 = *reinterpret_cast<const uint4 *>(prow + (((2 * j + half) ^ (r & 7)) << 4));
+          if (j == kSuperK - 1 || kb == nkb - 1) {
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&pk_empty[sp]);
+            if (++sp == C::kPkStages) {
+              sp = 0;
+              php ^= 1u;
+            }
+          }
+          const uint32_t wv[4] = {v0.x, v0.y, v0.z, v0.w};
+          uint32_t d[16];
+#pragma unroll
+          for (int cw = 0; cw < 4; ++cw) {
+            const uint4 v = dequant_word(wv[cw], s2, b2);
+            d[4 * cw + 0] = v.x;
+            d[4 * cw + 1] = v.y;
+            d[4 * cw + 2] = v.z;
+            d[4 * cw + 3] = v.w;
+          }
+          tmem_st_32x32b_x16(ta + 16 * half, d);
+        }
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&a_full[sa]);
-        if (++sa == kAStages) {
+        if (++sa == C::kAStages) {
           sa = 0;
           pha ^= 1u;
         }
