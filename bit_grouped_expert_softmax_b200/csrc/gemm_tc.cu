@@ -86,31 +86,6 @@ __device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volati
   return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
-// As warp_wait, but lane 0 sleeps between polls: for waits that usually last
-// a whole main loop, so the poll does not take issue slots from the dequant warps.
-__device__ __forceinline__ bool warp_wait_sleepy(uint64_t *bar, uint32_t parity, volatile int *abort,
-                                                 DevStatus *st, uint32_t site) {
-  int ok = 1;
-  if ((threadIdx.x & 31) == 0) {
-    const unsigned long long t0 = global_ns();
-    ok = 0;
-    while (true) {
-      if (mbar_try_wait(bar, parity)) {
-        ok = 1;
-        break;
-      }
-      if (*abort) break;
-      if (global_ns() - t0 > kWaitBudgetNs) {
-        *abort = 1;
-        report_error(st, kDevTimeout, site, blockIdx.x);
-        break;
-      }
-      __nanosleep(128);
-    }
-  }
-  return __shfl_sync(0xffffffffu, ok, 0) != 0;
-}
-
 // Wait (bounded, ignoring the abort flag) for the copies of the stages this
 // thread issued, before the CTA may exit.
 template <int N>
@@ -343,7 +318,7 @@ __global__ void __launch_bounds__(kThreads, 1) grouped_gemm_kernel(const GemmArg
       const bool sh = wi.group == a.E;
       const int st = li % C::kAccStages;
       const uint32_t acc_ph = (li / C::kAccStages) & 1;
-      if (!warp_wait_sleepy(&acc_full[st], acc_ph, abort, a.status, 120)) break;
+      if (!warp_wait(&acc_full[st], acc_ph, abort, a.status, 120)) break;
       tc_fence_after();
       const int mrow = wi.mblk * kTileM + q * 32 + lane;  // weight row of this thread
       const uint32_t tq = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + st * NMAT * kAccCols;
