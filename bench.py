@@ -332,6 +332,8 @@ def measured_traffic(kernel: str, workload: str):
         return None
     h = hashlib.sha256()
     for src in rec["sources"]:
+        if not os.path.exists(os.path.join(ROOT, src)):
+            return None
         with open(os.path.join(ROOT, src), "rb") as f:
             h.update(f.read())
     return rec["dram_bytes_per_launch"] if h.hexdigest()[:16] == rec["sha"] else None

@@ -59,7 +59,7 @@ int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 // Upper bounds of the two work lists for T tokens.
 int64_t max_gu_items(int64_t T, int64_t E, int64_t k, int64_t I, int64_t Is) {
   const int64_t R = T * k;
-  return (cdiv(R, kTileN) + std::min<int64_t>(E, R)) * (I / kTileM) + cdiv(T, kTileN) * (Is / kTileM);
+  return (cdiv(R, kGuTileN) + std::min<int64_t>(E, R)) * (I / kGuTileM) + cdiv(T, kGuTileN) * (Is / kGuTileM);
 }
 int64_t max_dn_items(int64_t T, int64_t E, int64_t k, int64_t H) {
   const int64_t R = T * k;

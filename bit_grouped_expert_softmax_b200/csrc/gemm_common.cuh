@@ -1,0 +1,125 @@
+// gemm_common.cuh -- pieces shared by the two grouped expert GEMMs (gate/up and
+// down): bounded warp waits, the teardown drain of in-flight copies, the
+// scale/bias row loads of the dequantisation warps and TMA descriptor set-up.
+#pragma once
+
+#include <cuda.h>
+
+#include "kernels.cuh"
+#include "sm100.cuh"
+
+namespace moe {
+namespace gemm {
+
+using namespace sm100;
+
+constexpr int kBRows = 32;  // TMA box height of activation rows
+
+struct alignas(64) TmaMaps {
+  CUtensorMap w;     // packed weights of the routed experts
+  CUtensorMap w_sh;  // packed weights of the shared expert
+  CUtensorMap b;     // activation rows (gate/up: gathered x; down: routed h)
+  CUtensorMap b_sh;  // down only: shared-expert h rows
+};
+
+// Lane 0 waits, the whole warp gets the outcome.
+__device__ __forceinline__ bool warp_wait(uint64_t *bar, uint32_t parity, volatile int *abort, DevStatus *st,
+                                          uint32_t site) {
+  int ok = 1;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abort, st, site) ? 1 : 0;
+  return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+// Wait (bounded, ignoring the abort flag) for the copies of the stages this
+// thread issued, before the CTA may exit.
+template <int N>
+__device__ __forceinline__ void drain_stages(uint64_t *full, uint32_t issued, uint32_t issued_ph) {
+  for (int t = 0; t < N; ++t) {
+    if (!(issued >> t & 1u)) continue;
+    const unsigned long long t0 = global_ns();
+    while (!mbar_try_wait(&full[t], issued_ph >> t & 1u) && global_ns() - t0 < kWaitBudgetNs) {
+    }
+  }
+}
+
+// 2^e as a float for |e| <= 126, built from its exponent bits
+__device__ __forceinline__ float pow2i(int e) { return __int_as_float((127 + e) << 23); }
+
+// The scale and bias row of one weight row, and its K extent.
+struct SbRow {
+  const uint16_t *S, *B;
+  int K;
+};
+
+// The scales and biases of K-blocks kb .. kb+3 of one row (bf16 bits, K-block
+// kb in the low half of .x); one 8-byte load each where the row allows it.
+__device__ __forceinline__ void load_sb4(const SbRow &w, int kb, uint2 &s, uint2 &b) {
+  const int nkb = w.K / kTileK;
+  if ((nkb & 3) == 0 && ((reinterpret_cast<uintptr_t>(w.S) | reinterpret_cast<uintptr_t>(w.B)) & 7) == 0) {
+    s = __ldg(reinterpret_cast<const uint2 *>(w.S + kb));
+    b = __ldg(reinterpret_cast<const uint2 *>(w.B + kb));
+  } else {
+    uint32_t sv[4], bv[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      sv[i] = kb + i < nkb ? __ldg(w.S + kb + i) : 0u;
+      bv[i] = kb + i < nkb ? __ldg(w.B + kb + i) : 0u;
+    }
+    s = make_uint2(sv[0] | sv[1] << 16, sv[2] | sv[3] << 16);
+    b = make_uint2(bv[0] | bv[1] << 16, bv[2] | bv[3] << 16);
+  }
+}
+
+__device__ __forceinline__ uint16_t pick_bf16(uint2 v, int j) {
+  const uint32_t w = (j & 2) ? v.y : v.x;
+  return static_cast<uint16_t>((j & 1) ? w >> 16 : w);
+}
+
+// Dequantise four packed words (32 weights of one row) into 16 fp16 pairs.
+__device__ __forceinline__ void dequant4(uint4 v, __half2 s2, __half2 b2, uint32_t (&d)[16]) {
+  const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+  for (int cw = 0; cw < 4; ++cw) {
+    const uint4 o = dequant_word(wv[cw], s2, b2);
+    d[4 * cw + 0] = o.x;
+    d[4 * cw + 1] = o.y;
+    d[4 * cw + 2] = o.z;
+    d[4 * cw + 3] = o.w;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host: tensor maps
+// ---------------------------------------------------------------------------
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                   const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+inline EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// rows x cols matrix, row-major; box = box_rows x box_cols elements
+inline bool make_map(CUtensorMap *m, CUtensorMapDataType dt, size_t elem, const void *base, uint64_t rows,
+                     uint64_t cols, uint32_t box_rows, uint32_t box_cols, CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * elem};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, dt, 2, const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace gemm
+}  // namespace moe

@@ -1,0 +1,411 @@
+// gemm_down.cu -- down projection of the grouped expert GEMM on the
+// 5th-generation tensor cores: Y = w_routing * (h W_down^T), per routed row.
+//
+// Same scheme as the gate/up GEMM: the 4-bit weights are rebuilt one tile at a
+// time on chip and the products accumulate in fp32 ("Perplexity open sources
+// Lily...", section "Measurements"; aioga.com record, article body paragraph
+// 4). The weights are the MMA's M side (128 rows of W_down) and the expert's
+// rows of h the N side (up to 128), so uneven expert groups, some with a
+// handful of tokens (aioga.com record, paragraph 3), only shrink N.
+//
+//   TMA: packed int4 rows (128-byte swizzle), fp16 h rows (32-row boxes)
+//   8 dequant warps: q*scale + bias -> fp16 -> TMEM (tcgen05.st), the MMA's A
+//   1 thread: tcgen05.mma (A from TMEM, B = h rows from shared memory)
+//   4 epilogue warps: tcgen05.ld, scale by the row's routing weight, fp16 rows
+//        of Y staged in shared memory and written out in 16-byte pieces.
+//
+// TMEM: two 128-column accumulator stages (a tile's epilogue overlaps the next
+// tile's main loop) and eight one-K-block weight stages of 32 columns.
+// Warp roles (480 threads): 0 weight TMA, 1 activation TMA, 2 MMA issue,
+// 3-6 epilogue, 7-14 dequantisation. Every wait is bounded.
+#include <algorithm>
+
+#include "gemm_common.cuh"
+
+namespace moe {
+
+namespace {
+
+using namespace sm100;
+using namespace gemm;
+
+constexpr int kThreads = 480;
+constexpr int kPkWarp = 0;
+constexpr int kBWarp = 1;
+constexpr int kMmaWarp = 2;
+constexpr int kEpiWarp0 = 3;
+constexpr int kDqWarp0 = 7;
+constexpr int kDqWarps = 8;
+
+constexpr int kN = kTileN;                     // activation rows per tile
+constexpr int kStageK = 2;                     // K-blocks per activation stage
+constexpr int kBStages = 3;
+constexpr int kBAtomBytes = kN * 128;          // one K-block of kN activation rows
+constexpr int kBStageBytes = kStageK * kBAtomBytes;
+constexpr int kSuperK = 4;                     // K-blocks per packed stage
+constexpr int kPkStages = 6;
+constexpr int kPkStageBytes = kTileM * 128;    // 128 weight rows x 32 words
+constexpr int kAStages = 8;                    // TMEM weight stages, one K-block (32 columns) each
+constexpr int kAccStages = 2;
+constexpr int kACol0 = kAccStages * kN;
+constexpr int kTmemCols = 512;
+static_assert(kACol0 + kAStages * 32 <= kTmemCols, "TMEM budget");
+constexpr int kStgBytes = kN * 32 * 2;         // per epilogue warp: kN rows x 32 columns fp16
+
+constexpr int kOffPk = 0;
+constexpr int kOffB = kOffPk + kPkStages * kPkStageBytes;
+constexpr int kOffStg = kOffB + kBStages * kBStageBytes;
+constexpr int kOffBar = kOffStg + 4 * kStgBytes;
+constexpr int kNumBars = 2 * kPkStages + 2 * kBStages + 2 * kAStages + 2 * kAccStages + 1;
+constexpr int kOffMisc = kOffBar + kNumBars * 8;
+constexpr int kSmem = kOffMisc + 64 + 1024;  // + slack for aligning the base
+static_assert(kOffB % 1024 == 0 && kBAtomBytes % 1024 == 0, "128-byte swizzle tiles need 1024-byte alignment");
+static_assert(kSmem <= 227 * 1024, "shared memory budget");
+
+// Scale/bias row of W_down row mblk*128 + r of item wi.
+__device__ __forceinline__ SbRow sb_row_dn(const GemmArgs &a, const WorkItem &wi, int r) {
+  const bool sh = wi.group == a.E;
+  const int Ig = sh ? a.Is : a.I;
+  const int H = a.H;
+  const size_t off = (sh ? 0 : static_cast<size_t>(wi.group) * 3 * a.I * H / kGroup) +
+                     static_cast<size_t>(2) * Ig * H / kGroup + static_cast<size_t>(wi.mblk * kTileM + r) * (Ig / kGroup);
+  return SbRow{(sh ? a.w.sh_scales : a.w.scales) + off, (sh ? a.w.sh_biases : a.w.biases) + off, Ig};
+}
+
+__global__ void __launch_bounds__(kThreads, 1) gemm_down_kernel(const GemmArgs a,
+                                                                const __grid_constant__ TmaMaps maps) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t *sPk = smem + kOffPk;
+  uint8_t *sB = smem + kOffB;
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBar);
+  uint64_t *pk_full = bars;
+  uint64_t *pk_empty = pk_full + kPkStages;
+  uint64_t *b_full = pk_empty + kPkStages;
+  uint64_t *b_empty = b_full + kBStages;
+  uint64_t *a_full = b_empty + kBStages;
+  uint64_t *a_empty = a_full + kAStages;
+  uint64_t *acc_full = a_empty + kAStages;
+  uint64_t *acc_empty = acc_full + kAccStages;
+  uint64_t *mma_done = acc_empty + kAccStages;
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kOffMisc);
+  volatile int *abort = reinterpret_cast<volatile int *>(smem + kOffMisc + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kPkStages; ++s) {
+      mbar_init(&pk_full[s], 1);
+      mbar_init(&pk_empty[s], kDqWarps);
+    }
+    for (int s = 0; s < kBStages; ++s) {
+      mbar_init(&b_full[s], 1);
+      mbar_init(&b_empty[s], 1);
+    }
+    for (int s = 0; s < kAStages; ++s) {
+      mbar_init(&a_full[s], kDqWarps);
+      mbar_init(&a_empty[s], 1);
+    }
+    for (int s = 0; s < kAccStages; ++s) {
+      mbar_init(&acc_full[s], 1);
+      mbar_init(&acc_empty[s], 4);  // four epilogue warps
+    }
+    mbar_init(mma_done, 1);
+    *abort = 0;
+    fence_barrier_init();
+    fence_proxy_async_smem();
+  }
+  if (warp == kMmaWarp) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == kPkWarp && lane == 0) {
+    tma_prefetch_desc(&maps.w);
+    tma_prefetch_desc(&maps.w_sh);
+  }
+  if (warp == kBWarp && lane == 0) {
+    tma_prefetch_desc(&maps.b);
+    tma_prefetch_desc(&maps.b_sh);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int nitems = min(*a.item_count, a.max_items);
+  const int H = a.H;
+
+  if (warp == kPkWarp) {
+    // ------------------------------------------------ producer: packed weights
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0, issued = 0, issued_ph = 0;
+      bool ok = true;
+      for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
+        const WorkItem wi = a.items[it];
+        const bool sh = wi.group == a.E;
+        const int K = sh ? a.Is : a.I;
+        // rows of K/8 words: an expert's block is 3H such rows, W_down its last H
+        const int wrow = (sh ? 0 : wi.group * 3 * H) + 2 * H + wi.mblk * kTileM;
+        const CUtensorMap *mw = sh ? &maps.w_sh : &maps.w;
+        for (int sb = 0; sb < (K / kTileK + kSuperK - 1) / kSuperK; ++sb) {
+          if (!mbar_wait(&pk_empty[s], ph ^ 1u, abort, a.status, 100)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&pk_full[s], kPkStageBytes);
+          issued |= 1u << s;
+          issued_ph = (issued_ph & ~(1u << s)) | (ph << s);
+          tma_load_2d(sPk + s * kPkStageBytes, mw, &pk_full[s], sb * kSuperK * 8, wrow);
+          if (++s == kPkStages) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+      if (!ok) drain_stages<kPkStages>(pk_full, issued, issued_ph);
+    }
+  } else if (warp == kBWarp) {
+    // ------------------------------------------------ producer: activation rows
+    if (lane == 0) {
+      int s = 0;
+      uint32_t ph = 0, issued = 0, issued_ph = 0;
+      bool ok = true;
+      for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
+        const WorkItem wi = a.items[it];
+        const bool sh = wi.group == a.E;
+        const int K = sh ? a.Is : a.I;
+        const CUtensorMap *mb = sh ? &maps.b_sh : &maps.b;
+        const int brow0 = sh ? wi.row0 - a.R : wi.row0;
+        const int nb = (wi.nrows + kBRows - 1) / kBRows;
+        for (int ks = 0; ks < K / (kTileK * kStageK); ++ks) {
+          if (!mbar_wait(&b_empty[s], ph ^ 1u, abort, a.status, 101)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&b_full[s], kStageK * nb * kBRows * 128);
+          issued |= 1u << s;
+          issued_ph = (issued_ph & ~(1u << s)) | (ph << s);
+#pragma unroll
+          for (int kh = 0; kh < kStageK; ++kh)
+            for (int j = 0; j < nb; ++j)
+              tma_load_2d(sB + s * kBStageBytes + kh * kBAtomBytes + j * kBRows * 128, mb, &b_full[s],
+                          (ks * kStageK + kh) * kTileK, brow0 + j * kBRows);
+          if (++s == kBStages) {
+            s = 0;
+            ph ^= 1u;
+          }
+        }
+      }
+      if (!ok) drain_stages<kBStages>(b_full, issued, issued_ph);
+    }
+  } else if (warp == kMmaWarp) {
+    // ------------------------------------------------ MMA issuer (whole warp, one elected lane issues)
+    int sb = 0, sa = 0;
+    uint32_t phb = 0, pha = 0;
+    bool ok = true;
+    int li = 0;
+    for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x, ++li) {
+      const WorkItem wi = a.items[it];
+      const int K = wi.group == a.E ? a.Is : a.I;
+      const int st = li % kAccStages;
+      const uint32_t acc_ph = (li / kAccStages) & 1;
+      if (!warp_wait(&acc_empty[st], acc_ph ^ 1u, abort, a.status, 110)) break;
+      tc_fence_after();
+      const uint32_t idesc = idesc_f16_f32(kTileM, (wi.nrows + 15) & ~15);
+      const uint32_t d = tmem_base + st * kN;
+      for (int ks = 0; ks < K / (kTileK * kStageK); ++ks) {
+        if (!warp_wait(&b_full[sb], phb, abort, a.status, 112)) {
+          ok = false;
+          break;
+        }
+        const uint32_t b_addr = smem_u32(sB + sb * kBStageBytes);
+        for (int kh = 0; kh < kStageK; ++kh) {
+          if (!warp_wait(&a_full[sa], pha, abort, a.status, 111)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (elect_one()) {
+            const uint32_t a_col = tmem_base + kACol0 + sa * 32;
+#pragma unroll
+            for (int kk = 0; kk < kTileK / 16; ++kk)
+              tc_mma_f16_ts(d, a_col + kk * 8, smem_desc_sw128(b_addr + kh * kBAtomBytes + kk * 32), idesc,
+                            (ks | kh | kk) != 0 ? 1u : 0u);
+            tc_commit(&a_empty[sa]);
+            if (kh == kStageK - 1) tc_commit(&b_empty[sb]);
+          }
+          __syncwarp();
+          if (++sa == kAStages) {
+            sa = 0;
+            pha ^= 1u;
+          }
+        }
+        if (!ok) break;
+        if (++sb == kBStages) {
+          sb = 0;
+          phb ^= 1u;
+        }
+      }
+      if (ok && elect_one()) tc_commit(&acc_full[st]);
+      __syncwarp();
+    }
+    // all issued MMAs finish before tensor memory is released
+    if (elect_one()) tc_commit(mma_done);
+    __syncwarp();
+    if (lane == 0) {
+      const unsigned long long t0 = global_ns();
+      while (!mbar_try_wait(mma_done, 0) && global_ns() - t0 < kWaitBudgetNs) {
+      }
+    }
+    __syncwarp();
+  } else if (warp < kDqWarp0) {
+    // ------------------------------------------------ epilogue
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    // this warp's 32 output columns of the tile's rows, staged as [row][32] fp16
+    __half *stg = reinterpret_cast<__half *>(smem + kOffStg + (warp - kEpiWarp0) * kStgBytes);
+    int li = 0;
+    for (int it = blockIdx.x; it < nitems; it += gridDim.x, ++li) {
+      const WorkItem wi = a.items[it];
+      const int st = li % kAccStages;
+      const uint32_t acc_ph = (li / kAccStages) & 1;
+      if (!warp_wait(&acc_full[st], acc_ph, abort, a.status, 120)) break;
+      tc_fence_after();
+      const uint32_t tq = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + st * kN;
+      __half *obase = a.y + static_cast<int64_t>(wi.row0) * H + wi.mblk * kTileM + q * 32;
+      for (int c0 = 0; c0 < wi.nrows; c0 += 32) {
+        // routing weight of each row, one row per lane, broadcast by shuffles
+        const int jl = c0 + lane;
+        const float wl = jl < wi.nrows ? a.row_w[wi.row0 + jl] : 0.f;
+        uint32_t r0[32];
+        tmem_ld_32x32b_x32(tq + c0, r0);
+        tmem_ld_wait();
+        if (c0 + 32 >= wi.nrows) {  // accumulators fully read: the next tile's MMAs may start
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[st]);
+        }
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) {
+          const float f = __shfl_sync(0xffffffffu, wl, jj);
+          stg[(c0 + jj) * 32 + lane] = __float2half_rn(f * __uint_as_float(r0[jj]));
+        }
+      }
+      __syncwarp();
+      // write out: 4 chunks of 16 bytes per row, 8 rows per warp instruction
+      for (int j = lane >> 2; j < wi.nrows; j += 8) {
+        const int c = lane & 3;
+        const uint4 v = *reinterpret_cast<const uint4 *>(stg + j * 32 + c * 8);
+        *reinterpret_cast<uint4 *>(obase + static_cast<int64_t>(j) * H + c * 8) = v;
+      }
+      __syncwarp();
+    }
+  } else {
+    // ------------------------------------------------ dequantisation
+    // Warp w owns TMEM lane quarter w % 4, i.e. weight rows 32*(w%4) + lane; the
+    // two warps of a quarter take four of the eight words of each row and
+    // K-block. The fp16 values go straight to TMEM (tcgen05.st), where the MMA
+    // reads its A operand.
+    const int dw = warp - kDqWarp0;
+    const int q = warp & 3;
+    const int r = q * 32 + lane;
+    const int half = dw >> 2;  // words 4*half .. 4*half+3 of each K-block
+    int sp = 0, sa = 0;
+    uint32_t php = 0, pha = 0;
+    bool ok = true;
+    // scales and biases: four K-blocks per load, one packed stage ahead; the
+    // first stage of the next item is fetched during the last stage of this one
+    SbRow row{};
+    uint2 s_cur{}, b_cur{}, s_nxt{}, b_nxt{};
+    if (blockIdx.x < nitems) {
+      row = sb_row_dn(a, a.items[blockIdx.x], r);
+      load_sb4(row, 0, s_nxt, b_nxt);
+    }
+    for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
+      const int nkb = row.K / kTileK;
+      SbRow next_row = row;
+      for (int kb = 0; kb < nkb; ++kb) {
+        const int j = kb % kSuperK;
+        if (j == 0) {
+          s_cur = s_nxt;
+          b_cur = b_nxt;
+          if (kb + kSuperK < nkb) {
+            load_sb4(row, kb + kSuperK, s_nxt, b_nxt);
+          } else if (it + static_cast<int>(gridDim.x) < nitems) {
+            next_row = sb_row_dn(a, a.items[it + gridDim.x], r);
+            load_sb4(next_row, 0, s_nxt, b_nxt);
+          }
+        }
+        if (!warp_wait(&a_empty[sa], pha ^ 1u, abort, a.status, 131)) {
+          ok = false;
+          break;
+        }
+        const __half2 s2 = bf16_to_half2_bcast(pick_bf16(s_cur, j));
+        const __half2 b2 = bf16_to_half2_bcast(pick_bf16(b_cur, j));
+        if (j == 0 && !warp_wait(&pk_full[sp], php, abort, a.status, 130)) {
+          ok = false;
+          break;
+        }
+        // row r of the packed stage: 128 bytes = 4 K-blocks of 8 words, in
+        // 16-byte chunks placed at chunk ^ (r & 7) by the TMA's 128-byte swizzle
+        const uint8_t *prow = sPk + sp * kPkStageBytes + r * 128;
+        const uint4 v0 = *reinterpret_cast<const uint4 *>(prow + (((2 * j + half) ^ (r & 7)) << 4));
+        if (j == kSuperK - 1 || kb == nkb - 1) {  // words in registers: release the packed stage
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&pk_empty[sp]);
+          if (++sp == kPkStages) {
+            sp = 0;
+            php ^= 1u;
+          }
+        }
+        uint32_t dq[16];
+        dequant4(v0, s2, b2, dq);
+        tmem_st_32x32b_x16(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + kACol0 + sa * 32 + 16 * half, dq);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&a_full[sa]);
+        if (++sa == kAStages) {
+          sa = 0;
+          pha ^= 1u;
+        }
+      }
+      row = next_row;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == kMmaWarp) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, kTmemCols);
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_down(const GemmArgs &a, int num_sms, cudaStream_t s) {
+  if (a.max_items <= 0) return cudaSuccess;
+  TmaMaps maps;
+  const int H = a.H;
+  bool ok = make_map(&maps.w, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, a.w.packed, static_cast<uint64_t>(a.E) * 3 * H,
+                     a.I / 8, kTileM, 32, CU_TENSOR_MAP_SWIZZLE_128B);
+  ok = ok && make_map(&maps.w_sh, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, a.w.sh_packed, static_cast<uint64_t>(3) * H,
+                      a.Is / 8, kTileM, 32, CU_TENSOR_MAP_SWIZZLE_128B);
+  ok = ok && make_map(&maps.b, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.h, static_cast<uint64_t>(a.h_rows), a.I, kBRows,
+                      kTileK, CU_TENSOR_MAP_SWIZZLE_128B);
+  ok = ok && make_map(&maps.b_sh, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.h + a.h_shared_off,
+                      static_cast<uint64_t>(a.hs_rows), a.Is, kBRows, kTileK, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!ok) return cudaErrorInvalidValue;
+  static bool configured = false;
+  if (!configured) {
+    const cudaError_t e = cudaFuncSetAttribute(gemm_down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  const int grid = std::max(1, std::min(num_sms, a.max_items));
+  gemm_down_kernel<<<grid, kThreads, kSmem, s>>>(a, maps);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -5,9 +5,11 @@
 
 namespace moe {
 
-constexpr int kTileM = 128;  // weight rows per grouped-GEMM tile (MMA M)
-constexpr int kTileN = 128;  // activation rows per grouped-GEMM tile (MMA N, max)
-constexpr int kTileK = 64;   // K elements per pipeline stage (one 128-byte fp16 row)
+constexpr int kTileM = 128;   // down GEMM: weight rows per tile (MMA M)
+constexpr int kTileN = 128;   // down GEMM: activation rows per tile (MMA N, max)
+constexpr int kGuTileM = 128; // gate/up GEMM: output rows per tile (the same rows of W_gate and W_up)
+constexpr int kGuTileN = 128; // gate/up GEMM: activation rows per tile (MMA N, max)
+constexpr int kTileK = 64;    // K elements per pipeline stage (one 128-byte fp16 row)
 
 struct RouteScanArgs {
   int T, E, k, H, I, Is, nchunk;

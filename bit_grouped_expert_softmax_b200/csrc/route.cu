@@ -79,9 +79,8 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(RouteScanArgs a) {
       int n = 0, gi = 0, di = 0;
       if (g < G) {
         n = (g < E) ? tot[g] : a.T;
-        const int ntile = (n + kTileN - 1) / kTileN;
-        gi = ntile * ((g < E ? a.I : a.Is) / kTileM);
-        di = ntile * (a.H / kTileM);
+        gi = ((n + kGuTileN - 1) / kGuTileN) * ((g < E ? a.I : a.Is) / kGuTileM);
+        di = ((n + kTileN - 1) / kTileN) * (a.H / kTileM);
       }
       cnt[i] = (g < E) ? n : 0;
       gu[i] = gi;
@@ -142,12 +141,12 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(RouteScanArgs a) {
     const int lane = threadIdx.x & 31;
     const int n = (g < E) ? tot[g] : a.T;
     const int row0 = (g < E) ? off[g] : R;
-    const int ntile = (n + kTileN - 1) / kTileN;
-    const int mg = (g < E ? a.I : a.Is) / kTileM, md = a.H / kTileM;
-    for (int i = lane; i < ntile * mg; i += 32) {
+    const int ntg = (n + kGuTileN - 1) / kGuTileN, ntile = (n + kTileN - 1) / kTileN;
+    const int mg = (g < E ? a.I : a.Is) / kGuTileM, md = a.H / kTileM;
+    for (int i = lane; i < ntg * mg; i += 32) {
       const int nt = i / mg, mb = i % mg, slot = gu_off[g] + i;
       if (slot < a.max_gu)
-        a.gu_items[slot] = WorkItem{g, row0 + nt * kTileN, min(kTileN, n - nt * kTileN), mb};
+        a.gu_items[slot] = WorkItem{g, row0 + nt * kGuTileN, min(kGuTileN, n - nt * kGuTileN), mb};
     }
     for (int i = lane; i < ntile * md; i += 32) {
       const int nt = i / md, mb = i % md, slot = dn_off[g] + i;
