@@ -2,20 +2,30 @@
 
     python -m bit_grouped_expert_softmax_b200.ncu_summary launches <launches.csv> [--skip-prefix at::]
     python -m bit_grouped_expert_softmax_b200.ncu_summary report <raw.csv>
+    python -m bit_grouped_expert_softmax_b200.ncu_summary record <raw.csv> <kernel-regex> <name> <workload> <summary.md> <source>...
 
 `launches` reads a `--metrics gpu__time_duration.sum --csv` launch list and
 prints, per kernel, the launch count, total and average device time and the
 share of the total. `report` reads `ncu -i <rep> --page raw --csv` and prints
 the counters used for the roofline (DRAM bytes and throughput, tensor-pipe
 activity, issue activity, registers, the largest warp-stall reasons).
+`record` stores one kernel's DRAM bytes per launch (read + write, averaged over
+the captured launches) in profiles/traffic.json under <name>, with the hash of
+the listed source files: bench.py reports the figure only while those sources
+are unchanged.
 """
 
 from __future__ import annotations
 
 import collections
 import csv
+import hashlib
+import json
+import os
 import re
 import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 _UNITS = {"ns": 1e-3, "nsecond": 1e-3, "us": 1.0, "usecond": 1.0, "ms": 1e3, "msecond": 1e3, "s": 1e6, "second": 1e6}
 
@@ -94,8 +104,41 @@ def report(path: str, top_stalls: int = 6) -> str:
     return "\n".join(out)
 
 
+def _num(v: str) -> float:
+    return float(v.replace(",", ""))
+
+
+_BYTES = {"byte": 1.0, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9}
+
+
+def record(path: str, kernel_re: str, name: str, workload: str, summary: str, sources: list[str]) -> dict:
+    rows = _rows(path)
+    h, units, data = rows[0], rows[1], rows[2:]
+    ki = h.index("Kernel Name")
+    ri, wi = h.index("dram__bytes_read.sum"), h.index("dram__bytes_write.sum")
+    per = [_num(d[ri]) * _BYTES[units[ri]] + _num(d[wi]) * _BYTES[units[wi]]
+           for d in data if re.search(kernel_re, d[ki])]
+    if not per:
+        raise SystemExit(f"no launch of {kernel_re} in {path}")
+    hs = hashlib.sha256()
+    for src in sources:
+        with open(os.path.join(ROOT, src), "rb") as f:
+            hs.update(f.read())
+    tpath = os.path.join(ROOT, "profiles", "traffic.json")
+    rec = json.load(open(tpath)) if os.path.exists(tpath) else {}
+    rec[name] = {"workload": workload, "dram_bytes_per_launch": int(round(sum(per) / len(per))),
+                 "sources": sources, "sha": hs.hexdigest()[:16], "from": summary}
+    with open(tpath, "w") as f:
+        json.dump(rec, f, indent=1)
+        f.write("\n")
+    return rec[name]
+
+
 if __name__ == "__main__":
-    if len(sys.argv) < 3 or sys.argv[1] not in ("launches", "report"):
+    if len(sys.argv) < 3 or sys.argv[1] not in ("launches", "report", "record"):
         print(__doc__)
         sys.exit(2)
-    print(launches(sys.argv[2]) if sys.argv[1] == "launches" else report(sys.argv[2]))
+    if sys.argv[1] == "record":
+        print(record(sys.argv[2], sys.argv[3], sys.argv[4], sys.argv[5], sys.argv[6], sys.argv[7:]))
+    else:
+        print(launches(sys.argv[2]) if sys.argv[1] == "launches" else report(sys.argv[2]))
