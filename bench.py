@@ -383,20 +383,37 @@ def cpu_baseline(name, budget_s=15.0):
     import oracle
     inp = synth.make_workload(name)
     cores = oracle.max_threads()
-    n = min(inp.T, max(1, cores))
-    t0 = time.perf_counter()
-    oracle.moe_forward(inp, x=inp.x[:n], logits=inp.logits[:n])
-    dt = time.perf_counter() - t0
-    per_tok = dt / n
-    n2 = int(min(inp.T if inp.T > 1 else 10 ** 9, max(n, budget_s / per_tok)))
-    xs = np.resize(inp.x, (n2, inp.H)) if n2 > inp.T else inp.x[:n2]
-    ls = np.resize(inp.logits, (n2, inp.E)) if n2 > inp.T else inp.logits[:n2]
-    t0 = time.perf_counter()
-    oracle.moe_forward(inp, x=np.ascontiguousarray(xs), logits=np.ascontiguousarray(ls))
-    dt = time.perf_counter() - t0
-    return {"value": round(n2 / dt, 3), "unit": "tokens/s", "cores": cores, "kind": "oracle",
-            "sample": f"{n2} tokens of the {name} layer (token rows repeated if T is smaller), fp64, "
-                      f"{dt:.1f} s wall"}
+
+    def rows(n):  # the workload's first n token rows, repeated if T is smaller
+        xs = np.resize(inp.x, (n, inp.H)) if n > inp.T else inp.x[:n]
+        ls = np.resize(inp.logits, (n, inp.E)) if n > inp.T else inp.logits[:n]
+        return np.ascontiguousarray(xs), np.ascontiguousarray(ls)
+
+    # grow the sample until one run takes about the budget (each call dequantises
+    # its touched experts once, so small samples cost more per token)
+    n2, dt = max(4 * cores, 8), 0.0
+    cap = max(inp.T, 1) if inp.T > 1 else 1 << 20
+    for _ in range(6):
+        n2 = min(n2, cap)
+        xs, ls = rows(n2)
+        t0 = time.perf_counter()
+        oracle.moe_forward(inp, x=xs, logits=ls)
+        dt = time.perf_counter() - t0
+        if dt >= 0.5 * budget_s or n2 >= cap:
+            break
+        n2 = int(n2 * min(8.0, budget_s / max(dt, 1e-3)))
+    out = {"value": round(n2 / dt, 3), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+           "sample": f"{n2} tokens of the {name} layer (token rows repeated if T is smaller), fp64, "
+                     f"{dt:.1f} s wall"}
+    if inp.T <= 512:
+        # the same rows on one core, sized to about a quarter of the budget
+        n1 = int(max(1, min(n2, budget_s / 4 / max(dt * cores / n2, 1e-9))))
+        t0 = time.perf_counter()
+        oracle.moe_forward(inp, nthreads=1, x=np.ascontiguousarray(xs[:n1]), logits=np.ascontiguousarray(ls[:n1]))
+        dt1 = time.perf_counter() - t0
+        out["single_core"] = {"value": round(n1 / dt1, 3), "unit": "tokens/s", "cores": 1,
+                              "sample": f"first {n1} of those tokens, {dt1:.1f} s wall"}
+    return out
 
 
 def main():

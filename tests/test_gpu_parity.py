@@ -125,6 +125,13 @@ def test_forward_small_batches(T, flags):
     check_output(_forward(_plan(inp, flags=flags), inp), oracle.moe_forward(inp), f"T={T} flags={flags}")
 
 
+@pytest.mark.parametrize("T,flags", [(1, 0), (4, 0), (4, api.MOE_FLAG_FORCE_GROUPED), (40, 0)])
+def test_shared_expert_narrower_than_routed(T, flags):
+    """Is < I on both paths (the small-batch kernel sizes its stages by the wider of the two)."""
+    inp = synth.make_layer(T, 512, 32, 4, 384, 128, seed=200 + T, logit_std=1.0)
+    check_output(_forward(_plan(inp, flags=flags), inp), oracle.moe_forward(inp), f"Is<I T={T} flags={flags}")
+
+
 def test_one_expert_takes_every_token():
     inp = synth.make_layer(150, 256, 16, 2, 128, 128, seed=31)
     inp.logits[:, 3] += 100.0  # expert 3 is everyone's first choice; most experts get nothing
