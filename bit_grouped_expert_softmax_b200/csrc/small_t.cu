@@ -69,7 +69,11 @@ struct StLayout {
 __host__ __device__ inline StLayout st_layout(int H, int I, int Is, int T, int k) {
   StLayout L;
   L.Imax = I > Is ? I : Is;
-  L.ks = H / kGroup < 8 ? H / kGroup : 8;
+  // K is split over ks warps per 16-row block, each walking its slice in
+  // 16-word (128-element) blocks: ks is the largest power of two <= 8 (so the
+  // 16 warps form whole groups) whose slices are whole 128-element blocks.
+  L.ks = 8;
+  while (L.ks > 1 && (H / 128) % L.ks != 0) L.ks >>= 1;
   L.kw = H / L.ks;
   L.b_stage = static_cast<size_t>(2) * kRowBlock * (H / 2) + static_cast<size_t>(4) * kRowBlock * (H / kGroup) * 2;
   L.d_stage = static_cast<size_t>(kRowBlock) * (L.Imax / 2) + static_cast<size_t>(2) * kRowBlock * (L.Imax / kGroup) * 2;

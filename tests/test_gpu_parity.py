@@ -132,6 +132,14 @@ def test_shared_expert_narrower_than_routed(T, flags):
     check_output(_forward(_plan(inp, flags=flags), inp), oracle.moe_forward(inp), f"Is<I T={T} flags={flags}")
 
 
+@pytest.mark.parametrize("H", [256, 512, 1280])
+@pytest.mark.parametrize("T", [1, 3])
+def test_small_batch_hidden_sizes(H, T):
+    """Hidden sizes whose per-warp K slices of the small-batch kernel are 1, 2 and 5 blocks of 128."""
+    inp = synth.make_layer(T, H, 16, 2, 128, 256, seed=300 + H + T, logit_std=1.0)
+    check_output(_forward(_plan(inp), inp), oracle.moe_forward(inp), f"H={H} T={T}")
+
+
 def test_one_expert_takes_every_token():
     inp = synth.make_layer(150, 256, 16, 2, 128, 128, seed=31)
     inp.logits[:, 3] += 100.0  # expert 3 is everyone's first choice; most experts get nothing
