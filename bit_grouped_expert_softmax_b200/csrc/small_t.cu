@@ -404,10 +404,12 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs
   const int n_units = nrb_sh + (nU - 1) * (a.I / kRowBlock);
   const int my_units = blockIdx.x < n_units ? (n_units - 1 - blockIdx.x) / gridDim.x + 1 : 0;
   const bool has_dblk = blockIdx.x < n_dblk;
-  if (warp == 0) {
+  // the requests block their warp while many copies are outstanding, so the
+  // phase-1 units (needed first) and the down rows go out from two warps
+  if (warp == 0)
     for (int q = shared_first ? 1 : 0; q < min(my_units, L.nb); ++q) issue_b(q);
-    if (has_dblk) issue_d_range(0, min(nU, L.nd));
-  }
+  else if (warp == 1 && has_dblk)
+    issue_d_range(0, min(nU, L.nd));
   // stage the tokens: fp16 scaled by 2^-e in operand order; rows t >= T are zero
 #pragma unroll
   for (int i = 0; i < kXPer; ++i) {
