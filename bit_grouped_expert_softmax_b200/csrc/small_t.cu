@@ -404,12 +404,15 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs
   const int n_units = nrb_sh + (nU - 1) * (a.I / kRowBlock);
   const int my_units = blockIdx.x < n_units ? (n_units - 1 - blockIdx.x) / gridDim.x + 1 : 0;
   const bool has_dblk = blockIdx.x < n_dblk;
-  // the requests block their warp while many copies are outstanding, so the
-  // phase-1 units (needed first) and the down rows go out from two warps
-  if (warp == 0)
-    for (int q = shared_first ? 1 : 0; q < min(my_units, L.nb); ++q) issue_b(q);
-  else if (warp == 1 && has_dblk)
-    issue_d_range(0, min(nU, L.nd));
+  // the requests block their warp while many copies are outstanding, so each
+  // phase-1 unit (needed first) goes out from its own warp (2, 3, ...) and the
+  // down rows from warp 1, all in parallel
+  if (warp == 1) {
+    if (has_dblk) issue_d_range(0, min(nU, L.nd));
+  } else if (warp >= 2) {
+    const int q = (shared_first ? 1 : 0) + warp - 2;
+    if (q < min(my_units, L.nb)) issue_b(q);
+  }
   // stage the tokens: fp16 scaled by 2^-e in operand order; rows t >= T are zero
 #pragma unroll
   for (int i = 0; i < kXPer; ++i) {
