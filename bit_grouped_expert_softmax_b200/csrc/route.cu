@@ -4,14 +4,17 @@
 // as work kept inside one GPU command buffer (aioga.com record, article body
 // paragraph 5); the router itself scores every expert and keeps the top k
 // ("Perplexity open sources Lily...", section "Requirements and model layout").
-// Three kernels:
+// Four kernels:
 //   route_topk_kernel    softmax over E, warp top-k, renormalised weights,
 //                        per-chunk expert histogram
 //   route_scan_kernel    per-expert totals, exclusive scan (offsets), per-chunk
 //                        bases, and the grouped-GEMM work lists (block map)
 //   route_scatter_kernel stable permutation (experts ascending, tokens ascending
-//                        within an expert), its inverse, and the gather of the
-//                        activations into expert-contiguous fp16 rows
+//                        within an expert) and its inverse
+//   gather_kernel        each token's row, fp16 scaled by a power of two, copied
+//                        to its k routed rows and its shared-expert row (expert-
+//                        contiguous, the gate/up GEMM's activation operand), and
+//                        the per-row exponents and weights the epilogues use
 #include "kernels.cuh"
 #include "topk.cuh"
 
