@@ -5,6 +5,8 @@
 
 #include <cuda.h>
 
+#include <atomic>
+
 #include "kernels.cuh"
 #include "sm100.cuh"
 
@@ -106,6 +108,20 @@ inline EncodeTiledFn encode_fn() {
       fn = reinterpret_cast<EncodeTiledFn>(p);
   }
   return fn;
+}
+
+// Raises a kernel's dynamic shared-memory limit on the current device, once
+// per device (the attribute belongs to the device's context, not the process).
+template <typename Kernel>
+inline cudaError_t ensure_smem_limit(Kernel kernel, int bytes, std::atomic<uint64_t> &done_devices) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = dev < 64 ? (uint64_t(1) << dev) : 0;
+  if (bit && (done_devices.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && bit) done_devices.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
 }
 
 // rows x cols matrix, row-major; box = box_rows x box_cols elements

@@ -397,12 +397,9 @@ cudaError_t launch_gemm_down(const GemmArgs &a, int num_sms, cudaStream_t s) {
   ok = ok && make_map(&maps.b_sh, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.h + a.h_shared_off,
                       static_cast<uint64_t>(a.hs_rows), a.Is, kBRows, kTileK, CU_TENSOR_MAP_SWIZZLE_128B);
   if (!ok) return cudaErrorInvalidValue;
-  static bool configured = false;
-  if (!configured) {
-    const cudaError_t e = cudaFuncSetAttribute(gemm_down_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  static std::atomic<uint64_t> smem_set{0};
+  const cudaError_t e = ensure_smem_limit(gemm_down_kernel, kSmem, smem_set);
+  if (e != cudaSuccess) return e;
   const int grid = std::max(1, std::min(num_sms, a.max_items));
   gemm_down_kernel<<<grid, kThreads, kSmem, s>>>(a, maps);
   return cudaGetLastError();

@@ -413,13 +413,9 @@ cudaError_t launch_gemm_gate_up(const GemmArgs &a, int num_sms, cudaStream_t s) 
                       kTileK, CU_TENSOR_MAP_SWIZZLE_128B);
   maps.b_sh = maps.b;
   if (!ok) return cudaErrorInvalidValue;
-  static bool configured = false;
-  if (!configured) {
-    const cudaError_t e =
-        cudaFuncSetAttribute(gemm_gate_up_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  static std::atomic<uint64_t> smem_set{0};
+  const cudaError_t e = ensure_smem_limit(gemm_gate_up_kernel, kSmem, smem_set);
+  if (e != cudaSuccess) return e;
   const int grid = std::max(1, std::min(num_sms, a.max_items));
   gemm_gate_up_kernel<<<grid, kThreads, kSmem, s>>>(a, maps);
   return cudaGetLastError();
