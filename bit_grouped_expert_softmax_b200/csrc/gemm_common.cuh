@@ -90,6 +90,19 @@ __device__ __forceinline__ void dequant4(uint4 v, __half2 s2, __half2 b2, uint32
   }
 }
 
+// Dequantise eight packed words (one row's K-block of 64 weights) into 32 fp16 pairs.
+__device__ __forceinline__ void dequant8(uint4 v0, uint4 v1, __half2 s2, __half2 b2, uint32_t (&d)[32]) {
+  const uint32_t wv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+  for (int cw = 0; cw < 8; ++cw) {
+    const uint4 o = dequant_word(wv[cw], s2, b2);
+    d[4 * cw + 0] = o.x;
+    d[4 * cw + 1] = o.y;
+    d[4 * cw + 2] = o.z;
+    d[4 * cw + 3] = o.w;
+  }
+}
+
 // ---------------------------------------------------------------------------
 // host: tensor maps
 // ---------------------------------------------------------------------------

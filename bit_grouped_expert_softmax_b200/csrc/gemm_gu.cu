@@ -374,8 +374,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_gate_up_kernel(const GemmArg
           }
         }
         uint32_t dq[32];
-        dequant4(v0, s2, b2, *reinterpret_cast<uint32_t(*)[16]>(dq));
-        dequant4(v1, s2, b2, *reinterpret_cast<uint32_t(*)[16]>(dq + 16));
+        dequant8(v0, v1, s2, b2, dq);
         tmem_st_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + kACol0 + sa * kAStageCols + m * 32,
                            dq);
         tmem_st_wait();

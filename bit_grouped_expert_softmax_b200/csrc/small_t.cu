@@ -276,9 +276,9 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs
   // Phase-1 units are (expert, 16-row block), the shared expert's blocks first;
   // unit q of this CTA is global unit blockIdx.x + q * gridDim.x and uses ring
   // stage q % nb. A unit is six bulk copies (gate rows, up rows, their scales
-  // and biases) from lanes 0..5 of warp 0.
+  // and biases) from lanes 0..5 of the calling warp.
   const int units_per_round = kSTWarps / L.ks;
-  auto issue_b = [&](int q) {  // all lanes of warp 0
+  auto issue_b = [&](int q) {  // all lanes of one warp
     const int unit = blockIdx.x + q * gridDim.x;
     int e, rb;
     if (unit < nrb_sh) {
@@ -307,7 +307,7 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs
   };
   // Phase-2 stage u % nd holds expert u's down rows [n0, n0 + 16): three copies,
   // ten experts per warp-wide step.
-  auto issue_d_range = [&](int u0, int u1) {  // all lanes of warp 0
+  auto issue_d_range = [&](int u0, int u1) {  // all lanes of one warp
     const int n0 = blockIdx.x * kRowBlock;
     for (int ub = u0; ub < u1; ub += 10) {
       const int sub = lane / 3, l = lane % 3, u = ub + sub;
