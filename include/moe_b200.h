@@ -112,8 +112,10 @@ int64_t moe_plan_workspace_bytes(const moe_plan_t *plan);
  *   router_logits [T, E] float32 router scores (finite values).
  *   packed_w, scales, biases, shared_*: the layer's weights (layout above).
  *   out_bf16      [T, H] bfloat16 output; must not overlap x_bf16.
- * T <= 8 runs the fused small-T kernel; larger T runs routing, gather,
- * grouped gate/up GEMM + SwiGLU, grouped down GEMM and the combine.
+ * T <= 8 runs the fused small-T kernel when the layer fits it (H a multiple
+ * of 256, H/16 no more than the GPU's SMs, its stages within shared memory);
+ * otherwise, and for larger T, routing, gather, grouped gate/up GEMM +
+ * SwiGLU, grouped down GEMM and the combine run.
  * Deterministic: the same inputs give bit-identical outputs.
  */
 moe_status moe_forward(moe_plan_t *plan, int T, const void *x_bf16,
@@ -194,7 +196,7 @@ moe_status moe_profile_read(moe_plan_t *plan, moe_stream_t stream, double *ms, i
 
 /*
  * The small-T layer (0 <= T <= 8 tokens) without any device allocation.
- * The paper has no counterpart to this call; it exists for callers that
+ * The source pages describe no such call; it exists for callers that
  * cannot call cudaMalloc (code running inside an allocator or memory-pool
  * callback, runtimes that reserve all device memory up front), and so cannot
  * create a plan. Its scratch memory (SwiGLU outputs, grid-barrier words,
