@@ -6,6 +6,9 @@ and it shares no code with the CUDA library.
 
 The arithmetic lives in ``moe_oracle.c`` (plain C, fp64, OpenMP over tokens);
 this module compiles it with gcc and marshals numpy arrays to it.
+``moe_forward_by_expert`` computes the same layer with the C routing and
+dequantisation and numpy's fp64 matrix products, so that every row of a
+full-size batch can be checked in seconds.
 """
 
 from __future__ import annotations
@@ -129,4 +132,64 @@ def moe_forward(inp, nthreads: int = 0, x: np.ndarray | None = None,
                                     *[_ptr(a) for a in args], _ptr(out), int(nthreads))
     if rc:
         raise ValueError("oracle_moe_forward: bad arguments")
+    return out
+
+
+def bf16_to_f64(bits: np.ndarray) -> np.ndarray:
+    """bfloat16 bit patterns -> exact float64 (the bits are the top half of a float32)."""
+    b = np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16
+    return b.view(np.float32).astype(np.float64)
+
+
+def moe_forward_by_expert(inp, x: np.ndarray | None = None, logits: np.ndarray | None = None,
+                          chunk: int = 2048) -> np.ndarray:
+    """The layer of ``moe_forward``, computed expert by expert (same definition).
+
+    Routing is the C oracle's. Each touched expert is dequantised once per
+    chunk of tokens into dense fp64 matrices (C ``oracle_dequant_matrix``:
+    w = q * scale + bias) and applied with fp64 matrix products to the tokens
+    routed to it: g = X Wg^T, u = X Wu^T, h = silu(g) * u, y = h Wd^T. Each
+    token's output is then summed in the fixed order j = 0..k-1 with its
+    renormalised routing weights, then the shared expert with weight 1. Only
+    the order of the additions inside a dot product differs from the per-token
+    C loop (the matrix product is a library routine), so the two agree to fp64
+    rounding.
+    """
+    x = _c(inp.x if x is None else x, np.uint16)
+    logits = _c(inp.logits if logits is None else logits, np.float32)
+    T, H, E, k, I, Is = x.shape[0], inp.H, inp.E, inp.k, inp.I, inp.Is
+    assert logits.shape == (T, E) and x.shape == (T, H)
+    out = np.empty((T, H), np.float64)
+    ids_all, w_all, _, _, _ = route(logits, k)
+
+    def expert_mats(words, scales, biases, Ie):
+        n1, g1 = Ie * H // 8, Ie * H // 64
+        wg = dequant_matrix(words[:n1], scales[:g1], biases[:g1], Ie, H)
+        wu = dequant_matrix(words[n1:2 * n1], scales[g1:2 * g1], biases[g1:2 * g1], Ie, H)
+        wd = dequant_matrix(words[2 * n1:], scales[2 * g1:], biases[2 * g1:], H, Ie)
+        return wg, wu, wd
+
+    def apply(mats, xs):
+        wg, wu, wd = mats
+        g = xs @ wg.T
+        u = xs @ wu.T
+        with np.errstate(over="ignore"):  # exp(-g) = inf for very negative g: silu -> 0
+            h = g / (1.0 + np.exp(-g)) * u  # silu(gate) * up
+        return h @ wd.T
+
+    for c0 in range(0, T, chunk):
+        c1 = min(T, c0 + chunk)
+        xs = bf16_to_f64(x[c0:c1])
+        ids, w = ids_all[c0:c1], w_all[c0:c1]
+        y = np.zeros((c1 - c0, k + 1, H), np.float64)  # per (token, slot) expert outputs
+        for e in np.unique(ids):
+            rows, slots = np.nonzero(ids == e)
+            mats = expert_mats(inp.packed[e], inp.scales[e], inp.biases[e], I)
+            y[rows, slots] = apply(mats, xs[rows])
+        y[:, k] = apply(expert_mats(inp.sh_packed, inp.sh_scales, inp.sh_biases, Is), xs)
+        o = np.zeros((c1 - c0, H), np.float64)
+        for j in range(k):
+            o += w[:, j:j + 1] * y[:, j]
+        o += y[:, k]  # shared expert, weight 1
+        out[c0:c1] = o
     return out

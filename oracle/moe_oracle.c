@@ -68,9 +68,12 @@ double oracle_weight(const uint32_t *words, const uint16_t *scales,
   return q * oracle_bf16_value(scales[g]) + oracle_bf16_value(biases[g]);
 }
 
-/* dequantise a whole N x K matrix into out[N*K] (fp64), for tests */
+/* dequantise a whole N x K matrix into out[N*K] (fp64); rows in parallel */
 void oracle_dequant_matrix(const uint32_t *words, const uint16_t *scales,
                            const uint16_t *biases, int N, int K, double *out) {
+#ifdef _OPENMP
+#pragma omp parallel for schedule(static)
+#endif
   for (int n = 0; n < N; ++n)
     for (int kk = 0; kk < K; ++kk)
       out[(size_t)n * K + kk] = oracle_weight(words, scales, biases, K, n, kk);

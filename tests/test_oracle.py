@@ -308,3 +308,32 @@ def test_thread_count_does_not_change_result():
 def test_empty_batch():
     inp = synth.make_workload("tiny", T=0)
     assert oracle.moe_forward(inp).shape == (0, inp.H)
+
+
+# ----------------------------------------------------------------------------
+# the by-expert form of the same layer (used to check every row at full size)
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("T,H,E,k,I,Is,chunk", [
+    (16, 256, 16, 2, 128, 128, 2048),   # the tiny layer, one chunk
+    (70, 512, 32, 4, 256, 384, 24),     # Is != I, several chunks with a ragged last one
+    (9, 256, 8, 8, 128, 64, 4),         # every expert routed (k = E), narrow shared expert
+])
+def test_by_expert_form_matches_per_token_oracle(T, H, E, k, I, Is, chunk):
+    inp = synth.make_layer(T, H, E, k, I, Is, seed=T + E, logit_std=1.0)
+    a = oracle.moe_forward(inp)
+    b = oracle.moe_forward_by_expert(inp, chunk=chunk)
+    scale = np.abs(a).max(axis=1, keepdims=True)
+    assert np.all(np.abs(a - b) <= 1e-12 * scale)
+
+
+def test_by_expert_form_matches_dense_brute_force_tiny():
+    inp = synth.make_workload("tiny")
+    out = oracle.moe_forward_by_expert(inp, chunk=5)
+    X = synth.bf16_to_f32(inp.x).astype(np.float64)
+    _, _, R = np_route_dense(inp.logits, inp.k)
+    want = np_swiglu_mlp(*np_expert_mats(inp.sh_packed, inp.sh_scales, inp.sh_biases, inp.H, inp.Is), X)
+    for e in range(inp.E):
+        Y = np_swiglu_mlp(*np_expert_mats(inp.packed[e], inp.scales[e], inp.biases[e], inp.H, inp.I), X)
+        want += R[:, e:e + 1] * Y
+    np.testing.assert_allclose(out, want, rtol=1e-10, atol=1e-10 * np.abs(want).max())
