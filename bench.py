@@ -1,14 +1,21 @@
 """Benchmark of the routed int4 MoE layer on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl b200|reference]
-                    [--workload decode|prefill|zipf|tiny] [--no-extra]
+                    [--workload decode|prefill|zipf|tiny|stack] [--no-extra]
+                    [--regions R] [--region-ms MS]
 
 One step = one MoE layer (routing, gate/up, down, combine) over one batch of
 synthetic inputs already resident in HBM. The headline workload is the decode
 layer (T=1, H=2048, E=256, top-8, I=Is=512); the prefill (T=512) and uneven
-Zipf (T=4096) layers are measured the same way and reported under "extra".
+Zipf (T=4096) layers and the 40-layer T=8192 stack are measured the same way
+and reported under "extra" (a stack step is one pass over all 40 layers).
 Weights rotate over device replicas whose touched bytes exceed 4x the L2, so
 every step reads its weights from HBM.
+
+Timing: a CUDA graph of consecutive steps is replayed until one timed region
+holds at least K steps and --region-ms of device time; R regions are timed
+with CUDA events on the launching stream and the median is reported
+("steps" = steps per region).
 
 Multi-GPU: one process per GPU; each rank runs its own batch (tokens are
 independent), no collective on the data path; value = all ranks' tokens over
@@ -147,6 +154,41 @@ def roofline_numbers(inp, peaks):
                 bound="hbm" if t_hbm >= t_tc else "tensor")
 
 
+def median_region_ms(run_region, regions, world, dev, stream, clk=None):
+    """Median over ``regions`` timed regions of one region's device time (CUDA
+    events on the launching stream, barrier + synchronize on both sides),
+    then the maximum of that median over the ranks."""
+    import torch
+    times = []
+    for _ in range(regions):
+        if world > 1:
+            torch.distributed.barrier()
+        torch.cuda.synchronize(dev)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        run_region()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        times.append(e0.elapsed_time(e1))
+    return reduce_max(statistics.median(times), world, dev), times
+
+
+def profile_kernels(api, plan, step, n_steps, stream, launches_per_step):
+    """Per-kernel device times of n_steps eager steps. The stream is first held
+    by a spin kernel long enough for the host to enqueue every step, so the
+    library's per-kernel CUDA events measure the kernels back to back on the
+    device and not the host's launch latency."""
+    import torch
+    api.moe_profile_enable(plan.handle, launches_per_step * n_steps + 8)
+    torch.cuda.synchronize()
+    torch.cuda._sleep(int(2e8))  # ~0.1 s at 2 GHz, on the current (launching) stream
+    for i in range(n_steps):
+        step(i)
+    prof = api.moe_profile_read(plan.handle, stream)
+    api.moe_profile_enable(plan.handle, 0)
+    return prof
+
+
 def run_gpu(args, rank, world, local_rank):
     import torch
     from bit_grouped_expert_softmax_b200 import api
@@ -157,7 +199,8 @@ def run_gpu(args, rank, world, local_rank):
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
 
     def measure_stack(steps, warmup):
-        """One step = the whole stack of layers over one T-token chunk."""
+        """One step = the whole stack of layers over one T-token chunk (x reset
+        from a device copy first, since the stack updates x in place)."""
         wl = synth.WORKLOADS["stack"]
         layers, logits, rfs = [], [], []
         for l in range(wl.layers):
@@ -165,16 +208,17 @@ def run_gpu(args, rank, world, local_rank):
             layers.append(api.DeviceLayer.from_inputs(inp, dev))
             logits.append(inp.logits)
             rfs.append(roofline_numbers(inp, peaks))
+            del inp
         rf = dict(rfs[0])
         rf["weight_bytes"] = sum(r["weight_bytes"] for r in rfs)
         rf["flops"] = sum(r["flops"] for r in rfs)
-        rf["touched"] = rfs[0]["touched"]
         rf["t_hbm"] = rf["weight_bytes"] / (peaks["hbm_gbs"] * 1e9)
         rf["t_tc"] = rf["flops"] / (peaks["bf16_tflops"] * 1e12)
         rf["bound"] = "hbm" if rf["t_hbm"] >= rf["t_tc"] else "tensor"
         x0 = torch.from_numpy(synth.make_stack_x(wl).view(np.int16)).to(dev)
         x = x0.clone()
         dlog = torch.from_numpy(np.stack(logits)).to(dev)
+        del logits
         plan = api.Plan(wl.T, wl.H, wl.E, wl.k, wl.I, wl.Is)
         stream = torch.cuda.Stream(dev)
         torch.cuda.set_stream(stream)
@@ -188,25 +232,32 @@ def run_gpu(args, rank, world, local_rank):
         plan.status_sync(stream)
         torch.cuda.synchronize(dev)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        with ClockSampler(local_rank) as clk:
-            e0.record(stream)
-            for i in range(steps):
+        e0.record(stream)
+        step(0)
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        per = max(e0.elapsed_time(e1), 1e-3)
+        n_steps = max(steps, int(np.ceil(args.region_ms / per)))
+
+        def region():
+            for i in range(n_steps):
                 step(i)
-            e1.record(stream)
-            torch.cuda.synchronize(dev)
-        ms_step = reduce_max(e0.elapsed_time(e1), world, dev) / steps
-        api.moe_profile_enable(plan.handle, 8 * wl.layers * 2)
-        for i in range(2):
-            step(i)
-        prof = api.moe_profile_read(plan.handle, stream)
-        api.moe_profile_enable(plan.handle, 0)
+
+        with ClockSampler(local_rank) as clk:
+            ms_region, all_regions = median_region_ms(region, args.regions, world, dev, stream)
         plan.status_sync(stream)
-        res = dict(workload="stack", T=wl.T, ms_per_step=ms_step, tokens_s=whole_job_tokens_s(wl.T, world, ms_step), rf=rf,
-                   achieved_gbs=rf["weight_bytes"] / (ms_step * 1e-3) / 1e9,
+        ms_step = ms_region / n_steps
+        prof = profile_kernels(api, plan, step, 1, stream, 7 * wl.layers)
+        plan.status_sync(stream)
+        res = dict(workload="stack", T=wl.T, ms_per_step=ms_step, tokens_s=whole_job_tokens_s(wl.T, world, ms_step),
+                   rf=rf, achieved_gbs=rf["weight_bytes"] / (ms_step * 1e-3) / 1e9,
                    achieved_tflops=rf["flops"] / (ms_step * 1e-3) / 1e12, n_rep=1, graph=False,
-                   timed_steps=steps, clocks=clk.summary(), e2e_tokens_s=None, h2d=0, d2h=0,
-                   launches=7 * wl.layers * steps, inp=None, prof=prof, layers=wl.layers)
+                   timed_steps=n_steps, regions=[round(t, 4) for t in all_regions], clocks=clk.summary(),
+                   e2e_tokens_s=None, h2d=0, d2h=0, launches=7 * wl.layers * n_steps, inp=None, prof=prof,
+                   layers=wl.layers, launches_per_step=7 * wl.layers)
         plan.close()
+        del layers, dlog
+        torch.cuda.empty_cache()
         return res
 
     def measure(name, steps, warmup):
@@ -222,96 +273,89 @@ def run_gpu(args, rank, world, local_rank):
         if args.replicas:
             n_rep = args.replicas
         reps = [base] + [api.DeviceLayer(*[t.clone() for t in base.args()]) for _ in range(n_rep - 1)]
+        rep_ptrs = [[t.data_ptr() for t in r.args()] for r in reps]
         x = torch.from_numpy(inp.x.view(np.int16)).to(dev)
         logits = torch.from_numpy(inp.logits).to(dev)
         out = torch.empty_like(x)
         plan = api.Plan(inp.T, inp.H, inp.E, inp.k, inp.I, inp.Is)
         stream = torch.cuda.Stream(dev)  # graphs cannot be captured on the default stream
         torch.cuda.set_stream(stream)
-        launches_per_step = 1 if inp.T <= 8 else 7
 
         def step(i):
-            api.moe_forward(plan.handle, inp.T, x, logits, *reps[i % n_rep].args(), out, stream)
+            api.moe_forward(plan.handle, inp.T, x, logits, *rep_ptrs[i % n_rep], out, stream)
 
         for i in range(warmup):
             step(i)
         plan.status_sync(stream)
-        # CUDA graph of n_rep consecutive steps (one pass over the replicas)
-        graph = None
-        try:
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
-                for i in range(n_rep):
-                    step(i)
-            g.replay()
-            torch.cuda.synchronize(dev)
-            plan.status_sync(stream)
-            graph = g
-        except Exception as e:  # capture unsupported: time eager launches
-            print(f"[bench] graph capture failed ({e}); timing eager launches", file=sys.stderr)
-            torch.cuda.synchronize(dev)
-        if world > 1:
-            torch.distributed.barrier()
-        torch.cuda.synchronize(dev)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        with ClockSampler(local_rank) as clk:
-            e0.record(stream)
-            if graph is not None:
-                reps_needed = -(-steps // n_rep)
-                for _ in range(reps_needed):
-                    graph.replay()
-                timed_steps = reps_needed * n_rep
-            else:
-                for i in range(steps):
-                    step(i)
-                timed_steps = steps
-            e1.record(stream)
-            torch.cuda.synchronize(dev)
-        ms = e0.elapsed_time(e1)
+        # per-kernel device times (and the number of launches one step makes)
+        prof = profile_kernels(api, plan, step, max(n_rep, 8), stream, 8)
         plan.status_sync(stream)
-        ms = reduce_max(ms, world, dev)
-        ms_step = ms / timed_steps
+        launches_per_step = max(1, round(sum(n for _, n in prof.values()) / max(n_rep, 8)))
+        # CUDA graph of n_rep consecutive steps (one pass over the replicas)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for i in range(n_rep):
+                step(i)
+        g.replay()
+        torch.cuda.synchronize(dev)
+        plan.status_sync(stream)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(4):
+            g.replay()
+        e1.record(stream)
+        torch.cuda.synchronize(dev)
+        per_replay = max(e0.elapsed_time(e1) / 4, 1e-4)
+        replays = max(-(-steps // n_rep), int(np.ceil(args.region_ms / per_replay)))
+        if world > 1:  # every rank replays the same number of times
+            replays = int(reduce_max(float(replays), world, dev))
+        timed_steps = replays * n_rep
+
+        def region():
+            for _ in range(replays):
+                g.replay()
+
+        with ClockSampler(local_rank) as clk:
+            ms_region, all_regions = median_region_ms(region, args.regions, world, dev, stream)
+        plan.status_sync(stream)
+        ms_step = ms_region / timed_steps
         tokens_s = whole_job_tokens_s(inp.T, world, ms_step)
         # end to end through the host-buffer entry point (pinned host memory)
         xh = torch.from_numpy(inp.x.view(np.int16)).pin_memory()
         lh = torch.from_numpy(inp.logits).pin_memory()
         oh = torch.empty_like(xh).pin_memory()
+        xp, lp, op = xh.data_ptr(), lh.data_ptr(), oh.data_ptr()
         for i in range(3):
-            api.moe_forward_host(plan.handle, inp.T, xh, lh, *reps[i % n_rep].args(), oh, stream)
-        n_e2e = max(10, min(200, steps))
+            api.moe_forward_host(plan.handle, inp.T, xp, lp, *rep_ptrs[i % n_rep], op, stream)
+        n_e2e = max(50, min(2000, int(0.2 / max(ms_step * 1e-3, 1e-6))))
         torch.cuda.synchronize(dev)
         t0 = time.perf_counter()
         for i in range(n_e2e):
-            api.moe_forward_host(plan.handle, inp.T, xh, lh, *reps[i % n_rep].args(), oh, stream)
+            api.moe_forward_host(plan.handle, inp.T, xp, lp, *rep_ptrs[i % n_rep], op, stream)
         e2e_s = (time.perf_counter() - t0) / n_e2e
-        plan.status_sync(stream)
-        # per-kernel times: the same steps launched eagerly with the library's
-        # CUDA events around every kernel, on the launching stream
-        api.moe_profile_enable(plan.handle, 8 * max(steps, n_rep))
-        torch.cuda.synchronize(dev)
-        for i in range(max(steps, n_rep)):
-            step(i)
-        prof = api.moe_profile_read(plan.handle, stream)
-        api.moe_profile_enable(plan.handle, 0)
+        e2e_s = reduce_max(e2e_s, world, dev)
         plan.status_sync(stream)
         achieved_gbs = rf["weight_bytes"] / (ms_step * 1e-3) / 1e9
         achieved_tf = rf["flops"] / (ms_step * 1e-3) / 1e12
         res = dict(workload=name, T=inp.T, ms_per_step=ms_step, tokens_s=tokens_s, rf=rf,
                    achieved_gbs=achieved_gbs, achieved_tflops=achieved_tf, n_rep=n_rep,
-                   graph=graph is not None, timed_steps=timed_steps, clocks=clk.summary(),
-                   e2e_tokens_s=inp.T * world / e2e_s,
+                   graph=True, timed_steps=timed_steps, regions=[round(t, 4) for t in all_regions],
+                   clocks=clk.summary(), e2e_tokens_s=inp.T * world / e2e_s,
                    h2d=inp.T * inp.H * 2 + inp.T * inp.E * 4, d2h=inp.T * inp.H * 2,
-                   launches=launches_per_step * timed_steps, inp=inp, prof=prof)
-        del graph
+                   launches=launches_per_step * timed_steps, inp=inp, prof=prof,
+                   launches_per_step=launches_per_step)
+        del g
         plan.close()
+        del reps, base
+        torch.cuda.empty_cache()
         return res
 
     main = measure(args.workload, args.steps, args.warmup)
     extra = {}
     if not args.no_extra and world == 1:
-        for name in ("prefill", "zipf"):
+        for name in ("prefill", "zipf", "stack"):
             if name != args.workload:
-                r = measure(name, max(10, args.steps // 4), args.warmup)
+                r = measure(name, 1 if name == "stack" else max(10, args.steps // 4), args.warmup)
                 extra[name] = summarize_extra(r, peaks, peaks_kind)
     return main, extra, peaks, peaks_kind
 
@@ -348,12 +392,21 @@ def kernel_table(r):
 
 def roofline_obj(r, peaks, peaks_kind):
     """Roofline of the dominant kernel: its algorithmic bytes or FLOPs per launch
-    over its average launch time (library CUDA events on the launch stream)."""
+    over its average launch duration.
+
+    A step of one launch (the small-batch kernel) takes the graph-timed step as
+    that duration, an upper bound of the kernel's own time. Otherwise the
+    duration is the library's per-kernel CUDA events on the launching stream,
+    recorded while the stream was pre-filled, so no host launch gap is counted."""
     rf = r["rf"]
     prof = r["prof"]
     name = max(prof, key=lambda k: prof[k][0])
     ms, n = prof[name]
     avg_s = ms * 1e-3 / max(n, 1)
+    timing = "per-kernel CUDA events on the pre-filled launching stream"
+    if r.get("launches_per_step") == 1:
+        avg_s = r["ms_per_step"] * 1e-3
+        timing = "CUDA-graph step time (one launch per step), median of the timed regions"
     fb, ff = KERNEL_SHARE.get(name, (0.0, 0.0))
     per_launch = 1.0 / r.get("layers", 1)  # the stack's totals cover every layer; a launch is one layer
     kbytes, kflops = rf["weight_bytes"] * fb * per_launch, rf["flops"] * ff * per_launch
@@ -366,13 +419,14 @@ def roofline_obj(r, peaks, peaks_kind):
     return {"bound": bound, "achieved": round(a, 2), "peak": p, "unit": unit, "frac": round(a / p, 4),
             "traffic": measured_traffic(name, r["workload"]), "traffic_unit": "bytes per launch (ncu)",
             "peak_source": peaks_kind, "kernel": name, "kernel_avg_us": round(avg_s * 1e6, 3),
+            "kernel_timing": timing,
             "algorithmic_per_launch": {"weight_bytes": int(kbytes), "flops": kflops,
                                        "touched_experts_incl_shared": rf["touched"]}}
 
 
 def summarize_extra(r, peaks, peaks_kind):
-    return {"T": r["T"], "tokens_s": round(r["tokens_s"], 1), "ms_per_step": round(r["ms_per_step"], 5),
-            "effective_tflops": round(r["achieved_tflops"], 2), "achieved_weight_gbs": round(r["achieved_gbs"], 1),
+    return {"T": r["T"], "tokens_s": round(r["tokens_s"], 1), "ms_per_step": round(r["ms_per_step"], 6),
+            "steps": r["timed_steps"], "region_ms": r["regions"], "effective_tflops": round(r["achieved_tflops"], 2), "achieved_weight_gbs": round(r["achieved_gbs"], 1),
             "roofline": roofline_obj(r, peaks, peaks_kind), "kernels": kernel_table(r), "graph": r["graph"],
             "clocks": r["clocks"],
             "e2e_tokens_s": None if r["e2e_tokens_s"] is None else round(r["e2e_tokens_s"], 1)}
@@ -425,6 +479,8 @@ def main():
     ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "zipf", "tiny", "stack"])
     ap.add_argument("--no-extra", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--regions", type=int, default=5, help="timed regions; the median is reported")
+    ap.add_argument("--region-ms", type=float, default=100.0, help="minimum device time of one timed region")
     ap.add_argument("--replicas", type=int, default=0,
                     help="weight replicas to rotate over (default: enough to exceed 4x L2); for profiling runs")
     args = ap.parse_args()
@@ -484,7 +540,9 @@ def main():
                 "data": "synthetic", "config": dict(config, l2=(
                     f"weights rotate over {r['n_rep']} device replicas "
                     f"({r['n_rep']} x {r['rf']['weight_bytes'] / 1e6:.1f} MB touched > 4 x L2)"),
-                    graph=r["graph"]),
+                    graph=r["graph"], timed_regions=len(r["regions"]),
+                    timing=f"median of {len(r['regions'])} CUDA-graph regions of {r['timed_steps']} steps each"),
+                "region_ms": r["regions"],
                 "roofline": roofline_obj(r, peaks, peaks_kind),
                 "kernels": kernel_table(r),
                 "effective_tflops": round(r["achieved_tflops"], 3),

@@ -47,6 +47,32 @@ def test_roofline_of_a_tensor_bound_kernel_takes_its_share_of_the_flops():
     assert o["achieved"] == pytest.approx(rf["flops"] * 2 / 3 / 230e-6 / 1e12, rel=1e-3)
 
 
+def test_one_launch_step_takes_the_graph_timed_step_as_the_kernel_time():
+    """A step of one launch: the graph-timed step bounds the kernel's own time,
+    so the roofline uses it even where eager event times are longer."""
+    inp = synth.make_workload("decode")
+    rf = bench.roofline_numbers(inp, PEAKS)
+    r = {"rf": rf, "prof": {"small_t": (23.0, 1000)}, "workload": "decode", "launches_per_step": 1,
+         "ms_per_step": 0.0125}
+    o = bench.roofline_obj(r, PEAKS, "measured")
+    assert o["kernel_avg_us"] == pytest.approx(12.5)
+    assert o["achieved"] == pytest.approx(rf["weight_bytes"] / 12.5e-6 / 1e9, rel=1e-3)
+    assert "graph" in o["kernel_timing"]
+
+
+def test_stack_roofline_is_per_layer_launch():
+    """The stack's totals cover all its layers; one gate/up launch is one layer's."""
+    inp = synth.make_workload("zipf")
+    rf = dict(bench.roofline_numbers(inp, PEAKS))
+    rf["flops"] *= 40
+    rf["weight_bytes"] *= 40
+    r = {"rf": rf, "prof": {"gate_up": (0.230 * 40, 40), "down": (0.17 * 40, 40)}, "workload": "stack",
+         "layers": 40, "launches_per_step": 280, "ms_per_step": 20.0}
+    o = bench.roofline_obj(r, PEAKS, "measured")
+    assert o["algorithmic_per_launch"]["flops"] == pytest.approx(rf["flops"] / 40 * 2 / 3)
+    assert o["kernel_avg_us"] == pytest.approx(230.0)
+
+
 def _run(args, env_extra=None):
     env = dict(os.environ)
     env.update(env_extra or {})
