@@ -6,9 +6,9 @@
 // allocation API is not reachable from the thread that issues work. For them,
 // moe_forward_small_t_noalloc runs the fused small-T kernel (batches of at
 // most 8 tokens) with its scratch memory -- the per-token SwiGLU outputs, the
-// grid-barrier words and the device status word -- taken from one file-scope
-// __device__ array instead of a plan's workspace. The caller still passes all
-// inputs and outputs.
+// kernel's readiness counters and the device status word -- taken from one
+// file-scope __device__ array instead of a plan's workspace. The caller still
+// passes all inputs and outputs.
 //
 // The array is created when the library's module is loaded on a device and
 // stays until the process exits, on every GPU that loads the library.
@@ -27,24 +27,51 @@ using namespace moe;
 namespace {
 
 constexpr size_t kStaticScratchBytes = 512 * 1024;  // stated maximum
-constexpr size_t kHeaderBytes = 256;                // barrier words + status word
+constexpr size_t kSyncOff = 0;                      // readiness and exit counters of the kernel
+constexpr size_t kStatusOff = 1024;                 // DevStatus
+constexpr size_t kHeaderBytes = 1280;               // cleared before every launch
+constexpr size_t kHOff = kHeaderBytes;              // fp16 SwiGLU outputs, 8 * (top_k + 1) * max(I, Is)
 constexpr int kMaxDevices = 64;
+static_assert(kSmallTSyncWords * 4 <= kStatusOff - kSyncOff, "counters fit the header");
 
-// [0, 16): grid barrier {count, generation}; [16, 32): DevStatus;
-// [256, kStaticScratchBytes): fp32 SwiGLU outputs, T * (top_k + 1) * max(I, Is)
+// [0, 1024): the kernel's synchronisation counters; [1024, 1040): DevStatus;
+// [1280, kStaticScratchBytes): fp16 SwiGLU outputs by token and slot.
 static __device__ __align__(256) unsigned char g_small_t_scratch[kStaticScratchBytes];
 
 struct DeviceSlot {
-  std::once_flag once;
-  cudaError_t err = cudaSuccess;
+  bool ready = false;
   unsigned char *ptr = nullptr;  // device address of g_small_t_scratch on this device
   int num_sms = 0;
 };
 DeviceSlot g_slots[kMaxDevices];
+std::mutex g_slots_mu;
 
 moe_status fail(moe_status st, const char *msg) {
   set_last_error(msg);
   return st;
+}
+
+// The array's device address on the current device, looked up (with that
+// device current) on the first call that succeeds; a failed lookup is not
+// remembered, so a later call retries it.
+cudaError_t device_slot(int dev, DeviceSlot *&out) {
+  std::lock_guard<std::mutex> lock(g_slots_mu);
+  DeviceSlot &slot = g_slots[dev];
+  if (!slot.ready) {
+    unsigned char *ptr = nullptr;
+    int sms = 0;
+    cudaError_t err = cudaGetSymbolAddress(reinterpret_cast<void **>(&ptr), g_small_t_scratch);
+    if (err == cudaSuccess) err = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (err != cudaSuccess || !ptr) {
+      cudaGetLastError();  // clear the (non-sticky) error so the caller's next CUDA call does not see it
+      return err != cudaSuccess ? err : cudaErrorInvalidSymbol;
+    }
+    slot.ptr = ptr;
+    slot.num_sms = sms;
+    slot.ready = true;
+  }
+  out = &slot;
+  return cudaSuccess;
 }
 
 }  // namespace
@@ -57,19 +84,27 @@ extern "C" moe_status moe_forward_small_t_noalloc(int T, int hidden, int n_exper
                                                   moe_stream_t stream) {
   set_last_error("");
   if (T < 0 || T > kSmallT) return fail(MOE_ERR_INVALID_ARG, "T must be in [0, 8]");
-  if (hidden < 128 || hidden % 128 || hidden > 16384 || inter < 128 || inter % 128 || inter > 8192 ||
-      shared_inter < 128 || shared_inter % 128 || shared_inter > 8192)
-    return fail(MOE_ERR_INVALID_ARG, "hidden, inter and shared_inter must be positive multiples of 128");
+  if (hidden < 256 || hidden % 256 || hidden > 16384)
+    return fail(MOE_ERR_INVALID_ARG, "hidden must be a positive multiple of 256 (at most 16384)");
+  if (inter < 128 || inter % 128 || inter > 8192 || shared_inter < 128 || shared_inter % 128 || shared_inter > 8192)
+    return fail(MOE_ERR_INVALID_ARG, "inter and shared_inter must be positive multiples of 128 (at most 8192)");
   if (n_experts < 1 || n_experts > kMaxExperts || top_k < 1 || top_k > n_experts || top_k > kMaxTopK)
     return fail(MOE_ERR_INVALID_ARG, "need 1 <= top_k <= min(n_experts, 16) and n_experts <= 256");
   const size_t imax = static_cast<size_t>(inter > shared_inter ? inter : shared_inter);
-  const size_t h_bytes = static_cast<size_t>(kSmallT) * (top_k + 1) * imax * sizeof(float);
-  if (kHeaderBytes + h_bytes > kStaticScratchBytes)
-    return fail(MOE_ERR_UNSUPPORTED, "8 * (top_k + 1) * max(inter, shared_inter) * 4 bytes exceeds the 512 KiB "
-                                     "static scratch");
-  if (T == 0) return MOE_OK;
-  const void *ptrs[10] = {x_bf16, router_logits, packed_w, scales, biases, shared_packed_w, shared_scales,
-                          shared_biases, out_bf16, nullptr};
+  const size_t h_bytes = static_cast<size_t>(kSmallT) * (top_k + 1) * imax * sizeof(__half);
+  if (kHOff + h_bytes > kStaticScratchBytes)
+    return fail(MOE_ERR_UNSUPPORTED, "8 * (top_k + 1) * max(inter, shared_inter) * 2 bytes exceeds the 512 KiB "
+                                     "static scratch (less its 1280-byte header)");
+  if (status_out && (reinterpret_cast<uintptr_t>(status_out) & 15u))
+    return fail(MOE_ERR_INVALID_ARG, "status_out must be 16-byte aligned");
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (T == 0) {  // nothing to compute; the status of this call is OK
+    if (status_out && cudaMemsetAsync(status_out, 0, sizeof(DevStatus), s) != cudaSuccess)
+      return fail(MOE_ERR_CUDA, "clearing status_out failed");
+    return MOE_OK;
+  }
+  const void *ptrs[9] = {x_bf16, router_logits, packed_w, scales, biases, shared_packed_w, shared_scales,
+                         shared_biases, out_bf16};
   for (int i = 0; i < 9; ++i)
     if (!ptrs[i] || (reinterpret_cast<uintptr_t>(ptrs[i]) & 15u))
       return fail(MOE_ERR_INVALID_ARG, "tensor pointers must be non-NULL and 16-byte aligned");
@@ -79,19 +114,14 @@ extern "C" moe_status moe_forward_small_t_noalloc(int T, int hidden, int n_exper
   cudaError_t err = cudaGetDevice(&dev);
   if (err != cudaSuccess) return fail(MOE_ERR_NO_DEVICE, "no current CUDA device");
   if (dev < 0 || dev >= kMaxDevices) return fail(MOE_ERR_UNSUPPORTED, "device ordinal above 63");
-  DeviceSlot &slot = g_slots[dev];
-  // once per device, with that device current: the array's device address
-  std::call_once(slot.once, [&slot, dev]() {
-    slot.err = cudaGetSymbolAddress(reinterpret_cast<void **>(&slot.ptr), g_small_t_scratch);
-    if (slot.err == cudaSuccess) slot.err = cudaDeviceGetAttribute(&slot.num_sms, cudaDevAttrMultiProcessorCount, dev);
-  });
-  if (slot.err != cudaSuccess || !slot.ptr) return fail(MOE_ERR_CUDA, "cudaGetSymbolAddress of the static scratch failed");
-  if (!small_t_fits(T, hidden, top_k, inter, shared_inter, slot.num_sms))
-    return fail(MOE_ERR_UNSUPPORTED, "layer too large for the small-T kernel");
+  DeviceSlot *slot = nullptr;
+  if (device_slot(dev, slot) != cudaSuccess)
+    return fail(MOE_ERR_CUDA, "cudaGetSymbolAddress of the static scratch failed");
+  if (!small_t_fits(T, hidden, top_k, inter, shared_inter, slot->num_sms))
+    return fail(MOE_ERR_UNSUPPORTED, "layer too large for the small-T kernel (shared memory or hidden/16 > SMs)");
 
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  // the array keeps the previous call's contents: reset the barrier and status words
-  err = cudaMemsetAsync(slot.ptr, 0, kHeaderBytes, s);
+  // the array keeps the previous call's contents: clear the counters and the status word
+  err = cudaMemsetAsync(slot->ptr, 0, kHeaderBytes, s);
   if (err != cudaSuccess) return fail(MOE_ERR_CUDA, "clearing the static scratch header failed");
   SmallTArgs a;
   a.T = T; a.E = n_experts; a.k = top_k; a.H = hidden; a.I = inter; a.Is = shared_inter;
@@ -103,15 +133,17 @@ extern "C" moe_status moe_forward_small_t_noalloc(int T, int hidden, int n_exper
   a.w.sh_packed = shared_packed_w;
   a.w.sh_scales = static_cast<const uint16_t *>(shared_scales);
   a.w.sh_biases = static_cast<const uint16_t *>(shared_biases);
-  a.barrier = reinterpret_cast<uint32_t *>(slot.ptr);
-  a.status = reinterpret_cast<DevStatus *>(slot.ptr + 16);
-  a.hbuf = reinterpret_cast<float *>(slot.ptr + kHeaderBytes);
+  a.sync = reinterpret_cast<uint32_t *>(slot->ptr + kSyncOff);
+  a.status = reinterpret_cast<DevStatus *>(slot->ptr + kStatusOff);
+  a.hbuf = reinterpret_cast<__half *>(slot->ptr + kHOff);
   a.residual = nullptr;
   a.out = static_cast<uint16_t *>(out_bf16);
-  err = launch_small_t(a, slot.num_sms, s);
+  a.wait_ns = kWaitBudgetNs;
+  a.test_fault = 0;
+  err = launch_small_t(a, slot->num_sms, s);
   if (err != cudaSuccess) return fail(MOE_ERR_CUDA, "small-T kernel launch failed");
   if (status_out) {
-    err = cudaMemcpyAsync(status_out, slot.ptr + 16, sizeof(DevStatus), cudaMemcpyDeviceToDevice, s);
+    err = cudaMemcpyAsync(status_out, slot->ptr + kStatusOff, sizeof(DevStatus), cudaMemcpyDeviceToDevice, s);
     if (err != cudaSuccess) return fail(MOE_ERR_CUDA, "copying the device status failed");
   }
   return MOE_OK;

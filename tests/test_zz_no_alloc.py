@@ -3,9 +3,10 @@
 moe_forward_small_t_noalloc serves callers that cannot call cudaMalloc (an
 allocator callback, a pool that owns all device memory, a runtime that
 reserves every byte up front): it takes its scratch from a static device
-array inside the library. Its output must match moe_forward's within the
-tests' tolerance, on two calls in a row, whether this file runs alone in a
-fresh process or after the rest of the suite.
+array inside the library. Both entry points run the same deterministic
+kernel on the same inputs, so its output must equal moe_forward's bit for
+bit (which implies the tests' tolerance), on two calls in a row, whether this
+file runs alone in a fresh process or after the rest of the suite.
 """
 
 import ctypes
@@ -47,17 +48,21 @@ def test_noalloc_matches_plan_entry_point_twice():
         x, logits = to_device(inp)
         plan = api.Plan(inp.T, inp.H, inp.E, inp.k, inp.I, inp.Is)
         ref = torch.empty_like(x)
+        torch.cuda.synchronize()  # inputs were made on the default stream
         api.moe_forward(plan.handle, inp.T, x, logits, *layer.args(), ref, stream)
         plan.status_sync(stream)
         for call in range(2):
             out = torch.full_like(x, 0x7FC0)  # NaN pattern: every element must be written
             status = torch.full((4,), -1, dtype=torch.int32, device="cuda")
+            torch.cuda.synchronize()  # the fills run on the default stream, the call on `stream`
             rc = _noalloc(lib, inp, x, logits, layer, out, status, stream)
             assert rc == 0, api.moe_last_error()
             stream.synchronize()
             assert status.cpu().numpy()[0] == 0, "device status reports an error"
-            ok, rel, row = _close(out.cpu().numpy(), ref.cpu().numpy())
+            got, want = out.cpu().numpy(), ref.cpu().numpy()
+            ok, rel, row = _close(got, want)
             assert ok, f"T={inp.T} call {call}: rel-L1 {rel:.3e}, row-max {row:.3e}"
+            assert np.array_equal(got, want), f"T={inp.T} call {call}: not bit-identical to moe_forward"
         plan.close()
 
 
@@ -66,8 +71,24 @@ def test_noalloc_rejects_sizes_beyond_its_scratch():
     f = lib.moe_forward_small_t_noalloc
     f.argtypes = [ctypes.c_int] * 6 + [ctypes.c_void_p] * 11
     f.restype = ctypes.c_int
-    # 8 * (16 + 1) * 8192 * 4 bytes > 512 KiB
+    # 8 * (16 + 1) * 8192 * 2 bytes of fp16 outputs > 512 KiB
     rc = f(1, 2048, 64, 16, 8192, 512, *([None] * 11))
     assert rc == -2 and "512 KiB" in api.moe_last_error()
     rc = f(9, 2048, 256, 8, 512, 512, *([None] * 11))
     assert rc == -1
+    rc = f(1, 384, 16, 2, 128, 128, *([None] * 11))  # hidden must be a multiple of 256
+    assert rc == -1 and "256" in api.moe_last_error()
+
+
+def test_noalloc_empty_batch_writes_an_ok_status():
+    lib = api.load()
+    f = lib.moe_forward_small_t_noalloc
+    f.argtypes = [ctypes.c_int] * 6 + [ctypes.c_void_p] * 11
+    f.restype = ctypes.c_int
+    status = torch.full((4,), -1, dtype=torch.int32, device="cuda")
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    rc = f(0, 2048, 256, 8, 512, 512, *([None] * 9), status.data_ptr(), stream.cuda_stream)
+    assert rc == 0, api.moe_last_error()
+    stream.synchronize()
+    assert status.cpu().numpy().tolist() == [0, 0, 0, 0]
