@@ -24,6 +24,9 @@ STATUS_NAMES = {0: "MOE_OK", -1: "MOE_ERR_INVALID_ARG", -2: "MOE_ERR_UNSUPPORTED
 MOE_FLAG_NONE = 0
 MOE_FLAG_FORCE_GROUPED = 1
 MOE_FLAG_FORCE_SMALL_T = 2
+MOE_FLAG_DEBUG = 4
+MOE_FLAG_TEST_WAIT_TIMEOUT = 8
+MOE_FLAG_NO_PDL = 16
 
 _lib = None
 
@@ -55,6 +58,8 @@ def load():
     lib.moe_plan_workspace_bytes.restype = L
     lib.moe_forward.argtypes = [P, I, P, P, P, P, P, P, P, P, P, P]
     lib.moe_forward_host.argtypes = [P, I, P, P, P, P, P, P, P, P, P, P]
+    lib.moe_forward_router.argtypes = [P, I, P, P, P, P, P, P, P, P, P, P]
+    lib.moe_router_logits.argtypes = [P, I, P, P, P, P]
     lib.moe_stack_forward.argtypes = [P, I, I, P, P, ctypes.POINTER(moe_layer_weights), P]
     lib.moe_route.argtypes = [P, I, P, P, P, P, P, P]
     lib.moe_status_sync.argtypes = [P, P]
@@ -62,7 +67,8 @@ def load():
     lib.moe_profile_read.argtypes = [P, P, P, P]
     lib.moe_last_error.restype = ctypes.c_char_p
     lib.moe_version.restype = ctypes.c_char_p
-    for name in ("moe_plan", "moe_plan_destroy", "moe_forward", "moe_forward_host", "moe_stack_forward",
+    for name in ("moe_plan", "moe_plan_destroy", "moe_forward", "moe_forward_host", "moe_forward_router",
+                 "moe_router_logits", "moe_stack_forward",
                  "moe_route", "moe_status_sync", "moe_profile_enable", "moe_profile_read"):
         getattr(lib, name).restype = I
     _lib = lib
@@ -123,6 +129,17 @@ def moe_forward(plan, T, x, logits, packed_w, scales, biases, shared_packed_w, s
                               _stream(stream)))
 
 
+def moe_forward_router(plan, T, x, router_w, packed_w, scales, biases, shared_packed_w, shared_scales,
+                       shared_biases, out, stream=None):
+    _check(load().moe_forward_router(plan, T, _ptr(x), _ptr(router_w), _ptr(packed_w), _ptr(scales), _ptr(biases),
+                                     _ptr(shared_packed_w), _ptr(shared_scales), _ptr(shared_biases), _ptr(out),
+                                     _stream(stream)))
+
+
+def moe_router_logits(plan, T, x, router_w, logits_out, stream=None):
+    _check(load().moe_router_logits(plan, T, _ptr(x), _ptr(router_w), _ptr(logits_out), _stream(stream)))
+
+
 def moe_forward_host(plan, T, x_host, logits_host, packed_w, scales, biases, shared_packed_w, shared_scales,
                      shared_biases, out_host, stream=None):
     _check(load().moe_forward_host(plan, T, _ptr(x_host), _ptr(logits_host), _ptr(packed_w), _ptr(scales),
@@ -148,7 +165,8 @@ def moe_status_sync(plan, stream=None):
     _check(load().moe_status_sync(plan, _stream(stream)))
 
 
-KERNEL_NAMES = ["route_topk", "route_scan", "route_scatter", "gather", "gate_up", "down", "combine", "small_t"]
+KERNEL_NAMES = ["route_topk", "route_scan", "route_scatter", "gather", "gate_up", "down", "combine", "small_t",
+                "router"]
 
 
 def moe_profile_enable(plan, max_launches):

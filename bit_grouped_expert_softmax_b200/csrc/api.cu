@@ -86,16 +86,19 @@ struct moe_plan_s {
   WorkItem *gu_items;
   WorkItem *dn_items;
   int32_t *item_counts;
+  int32_t *scan_done;
   __half *xt;
   __half *h;
   __half *y;
-  float *hsmall;
+  __half *hsmall;
   DevStatus *status;
-  uint32_t *barrier;
+  uint32_t *small_sync;
   uint16_t *x_stage;
   float *logits_stage;
+  float *router_logits;  // [T_max, E] scores computed from a router weight
   uint16_t *out_stage;
   int64_t max_gu, max_dn;
+  bool test_fault_armed = false;  // MOE_FLAG_TEST_WAIT_TIMEOUT: the next small-T launch carries the fault
   // per-kernel timing (moe_profile_enable / moe_profile_read)
   std::vector<cudaEvent_t> prof_events;  // 2 per recorded launch
   std::vector<int> prof_kind;
@@ -148,6 +151,10 @@ LayerWeights make_weights(const void *packed, const void *scales, const void *bi
   return w;
 }
 
+// Whether the grouped path's kernels go out with programmatic dependent launch.
+// Not while profiling: the events between kernels would separate them anyway.
+bool pdl(const moe_plan_s *p) { return !(p->flags & MOE_FLAG_NO_PDL) && p->prof_kind.empty(); }
+
 // Brackets one kernel launch with the plan's profiling events, if enabled.
 struct ProfScope {
   moe_plan_s *p;
@@ -171,51 +178,77 @@ moe_status enqueue_routing(moe_plan_s *p, int T, const float *logits, const uint
   const int tok_blocks = static_cast<int>(cdiv(T, 8));
   {
     ProfScope ps(p, MOE_KERNEL_ROUTE_TOPK, s);
-    route_topk_kernel<<<tok_blocks, 256, 0, s>>>(T, p->E, p->k, logits, p->ids, p->wts, p->chunk);
-    MOE_CUDA(cudaGetLastError(), "route_topk launch");
+    MOE_CUDA(launch_k(route_topk_kernel, dim3(tok_blocks), dim3(256), 0, s, pdl(p), T, p->E, p->k, logits, p->ids,
+                      p->wts, p->chunk),
+             "route_topk launch");
   }
   RouteScanArgs sa;
   sa.T = T; sa.E = p->E; sa.k = p->k; sa.H = p->H; sa.I = p->I; sa.Is = p->Is; sa.nchunk = nchunk;
   sa.chunk_cnt = p->chunk; sa.offsets = p->offsets;
   sa.gu_items = p->gu_items; sa.max_gu = static_cast<int>(p->max_gu);
   sa.dn_items = p->dn_items; sa.max_dn = static_cast<int>(p->max_dn);
-  sa.item_counts = p->item_counts; sa.status = p->status;
+  sa.item_counts = p->item_counts; sa.done = p->scan_done; sa.status = p->status;
   {
     ProfScope ps(p, MOE_KERNEL_ROUTE_SCAN, s);
-    route_scan_kernel<<<1, 1024, 0, s>>>(sa);
-    MOE_CUDA(cudaGetLastError(), "route_scan launch");
+    MOE_CUDA(launch_k(route_scan_kernel, dim3(static_cast<int>(cdiv(p->E, 8))), dim3(256), 0, s, pdl(p), sa),
+             "route_scan launch");
   }
   RouteScatterArgs ca;
   ca.T = T; ca.E = p->E; ca.k = p->k; ca.H = p->H;
-  ca.ids = p->ids; ca.chunk_base = p->chunk; ca.perm = p->perm; ca.inv = p->inv;
+  ca.ids = p->ids; ca.chunk_base = p->chunk; ca.offsets = p->offsets; ca.perm = p->perm; ca.inv = p->inv;
   ca.x = x; ca.xt = p->xt; ca.xexp = p->xexp; ca.status = p->status;
   ca.wts = p->wts; ca.row_exp = p->row_exp; ca.row_w = p->row_w;
   {
     ProfScope ps(p, MOE_KERNEL_ROUTE_SCATTER, s);
-    route_scatter_kernel<<<nchunk, 256, 0, s>>>(ca);
-    MOE_CUDA(cudaGetLastError(), "route_scatter launch");
+    MOE_CUDA(launch_k(route_scatter_kernel, dim3(nchunk), dim3(256), 0, s, pdl(p), ca), "route_scatter launch");
   }
   if (x) {
     ProfScope ps(p, MOE_KERNEL_GATHER, s);
-    gather_kernel<<<tok_blocks, 256, 0, s>>>(ca);
-    MOE_CUDA(cudaGetLastError(), "gather launch");
+    MOE_CUDA(launch_k(gather_kernel, dim3(tok_blocks), dim3(256), 0, s, pdl(p), ca), "gather launch");
   }
   return MOE_OK;
 }
 
+// Router scores of T tokens into the plan's workspace (grouped path).
+moe_status enqueue_router(moe_plan_s *p, int T, const uint16_t *x, const uint16_t *router_w, float *logits,
+                          cudaStream_t s) {
+  RouterArgs r;
+  r.T = T; r.E = p->E; r.H = p->H; r.x = x; r.w = router_w; r.logits = logits; r.status = p->status;
+  ProfScope ps(p, MOE_KERNEL_ROUTER, s);
+  MOE_CUDA(launch_router(r, s, pdl(p)), "router launch");
+  return MOE_OK;
+}
+
+// One layer. With router_w set, the logits are computed from it (and the
+// logits argument is ignored): inside the small-T kernel, or by the router
+// kernel ahead of the grouped path's routing.
 moe_status enqueue_layer(moe_plan_s *p, int T, const uint16_t *x, const float *logits, const LayerWeights &w,
-                         const uint16_t *residual, uint16_t *out, cudaStream_t s) {
+                         const uint16_t *residual, uint16_t *out, cudaStream_t s,
+                         const uint16_t *router_w = nullptr) {
   if (T == 0) return MOE_OK;
   if (use_small_t(p, T) || (p->flags & MOE_FLAG_FORCE_SMALL_T)) {
     if (!small_t_fits(T, p->H, p->k, p->I, p->Is, p->num_sms))
       return fail(MOE_ERR_UNSUPPORTED, "small-T path needs T <= %d and a small enough layer", kSmallT);
     SmallTArgs a;
     a.T = T; a.E = p->E; a.k = p->k; a.H = p->H; a.I = p->I; a.Is = p->Is;
-    a.x = x; a.logits = logits; a.w = w; a.hbuf = p->hsmall; a.barrier = p->barrier;
+    a.x = x; a.logits = router_w ? p->router_logits : logits; a.router_w = router_w;
+    a.w = w; a.hbuf = p->hsmall; a.sync = p->small_sync;
     a.residual = residual; a.out = out; a.status = p->status;
+    a.wait_ns = kWaitBudgetNs;
+    a.test_fault = 0;
+    if (p->test_fault_armed) {  // one launch only
+      a.test_fault = 1;
+      a.wait_ns = kTestWaitBudgetNs;
+      p->test_fault_armed = false;
+    }
     ProfScope ps(p, MOE_KERNEL_SMALL_T, s);
     MOE_CUDA(launch_small_t(a, p->num_sms, s), "small-T kernel launch");
     return MOE_OK;
+  }
+  if (router_w) {
+    moe_status st = enqueue_router(p, T, x, router_w, p->router_logits, s);
+    if (st != MOE_OK) return st;
+    logits = p->router_logits;
   }
   moe_status st = enqueue_routing(p, T, logits, x, s);
   if (st != MOE_OK) return st;
@@ -225,6 +258,7 @@ moe_status enqueue_layer(moe_plan_s *p, int T, const uint16_t *x, const float *l
   g.h_shared_off = static_cast<int64_t>(p->T_max) * p->k * p->I;
   g.y = p->y; g.perm = p->perm; g.wts = p->wts; g.xexp = p->xexp; g.status = p->status;
   g.row_exp = p->row_exp; g.row_w = p->row_w;
+  g.debug = (p->flags & MOE_FLAG_DEBUG) ? 1 : 0;
   g.xt_rows = static_cast<int64_t>(p->T_max) * (p->k + 1);
   g.h_rows = static_cast<int64_t>(p->T_max) * p->k;
   g.hs_rows = p->T_max;
@@ -233,21 +267,22 @@ moe_status enqueue_layer(moe_plan_s *p, int T, const uint16_t *x, const float *l
   g.max_items = static_cast<int>(max_gu_items(T, p->E, p->k, p->I, p->Is));
   {
     ProfScope ps(p, MOE_KERNEL_GATE_UP, s);
-    MOE_CUDA(launch_gemm_gate_up(g, p->num_sms, s), "gate/up GEMM launch");
+    MOE_CUDA(launch_gemm_gate_up(g, p->num_sms, s, pdl(p)), "gate/up GEMM launch");
   }
   g.items = p->dn_items;
   g.item_count = p->item_counts + 1;
   g.max_items = static_cast<int>(max_dn_items(T, p->E, p->k, p->H));
   {
     ProfScope ps(p, MOE_KERNEL_DOWN, s);
-    MOE_CUDA(launch_gemm_down(g, p->num_sms, s), "down GEMM launch");
+    MOE_CUDA(launch_gemm_down(g, p->num_sms, s, pdl(p)), "down GEMM launch");
   }
   CombineArgs c;
   c.T = T; c.k = p->k; c.H = p->H; c.R = T * p->k;
   c.inv = p->inv; c.y = p->y; c.xexp = p->xexp; c.residual = residual; c.out = out;
+  c.status = p->status; c.debug = (p->flags & MOE_FLAG_DEBUG) ? 1 : 0;
   {
     ProfScope ps(p, MOE_KERNEL_COMBINE, s);
-    MOE_CUDA(launch_combine(c, s), "combine launch");
+    MOE_CUDA(launch_combine(c, s, pdl(p)), "combine launch");
   }
   return MOE_OK;
 }
@@ -269,7 +304,8 @@ moe_status moe_plan(int T_max, int hidden, int n_experts, int top_k, int inter, 
   if (st != MOE_OK) return st;
   if ((flags & MOE_FLAG_FORCE_GROUPED) && (flags & MOE_FLAG_FORCE_SMALL_T))
     return fail(MOE_ERR_INVALID_ARG, "flags FORCE_GROUPED and FORCE_SMALL_T exclude each other");
-  if (flags & ~(MOE_FLAG_FORCE_GROUPED | MOE_FLAG_FORCE_SMALL_T))
+  if (flags & ~(MOE_FLAG_FORCE_GROUPED | MOE_FLAG_FORCE_SMALL_T | MOE_FLAG_DEBUG | MOE_FLAG_TEST_WAIT_TIMEOUT |
+                MOE_FLAG_NO_PDL))
     return fail(MOE_ERR_INVALID_ARG, "unknown flags 0x%x", flags);
   int dev = 0, ndev = 0;
   if (cudaGetDeviceCount(&ndev) != cudaSuccess || ndev == 0) {
@@ -286,6 +322,7 @@ moe_status moe_plan(int T_max, int hidden, int n_experts, int top_k, int inter, 
   moe_plan_s *p = new moe_plan_s();
   p->T_max = T_max; p->H = hidden; p->E = n_experts; p->k = top_k; p->I = inter; p->Is = shared_inter;
   p->flags = flags; p->device = dev; p->num_sms = prop.multiProcessorCount;
+  p->test_fault_armed = (flags & MOE_FLAG_TEST_WAIT_TIMEOUT) != 0;
   p->max_gu = max_gu_items(T_max, n_experts, top_k, inter, shared_inter);
   p->max_dn = max_dn_items(T_max, n_experts, top_k, hidden);
   const size_t T = T_max, H = hidden, E = n_experts, k = top_k, I = inter, Is = shared_inter;
@@ -303,14 +340,16 @@ moe_status moe_plan(int T_max, int hidden, int n_experts, int top_k, int inter, 
       static_cast<size_t>(p->max_gu) * sizeof(WorkItem),
       static_cast<size_t>(p->max_dn) * sizeof(WorkItem),
       16,                                    // item counts
+      16,                                    // scan: blocks finished
       (R + T) * H * 2,                       // xt
       (R * I + T * Is) * 2,                  // h
       (R + T) * H * 2,                       // y
-      static_cast<size_t>(kSmallT) * (k + 1) * std::max(I, Is) * 4,  // small-T h
+      static_cast<size_t>(kSmallT) * (k + 1) * std::max(I, Is) * 2,  // small-T h (fp16)
       sizeof(DevStatus),                     // status
-      16,                                    // barrier
+      kSmallTSyncWords * 4,                  // small-T readiness and exit counters
       T * H * 2,                             // x staging
       T * E * 4,                             // logits staging
+      T * E * 4,                             // router scores
       T * H * 2,                             // out staging
   };
   constexpr int nbuf = sizeof(sizes) / sizeof(sizes[0]);
@@ -339,14 +378,16 @@ moe_status moe_plan(int T_max, int hidden, int n_experts, int top_k, int inter, 
   p->gu_items = reinterpret_cast<WorkItem *>(b + offs[i++]);
   p->dn_items = reinterpret_cast<WorkItem *>(b + offs[i++]);
   p->item_counts = reinterpret_cast<int32_t *>(b + offs[i++]);
+  p->scan_done = reinterpret_cast<int32_t *>(b + offs[i++]);
   p->xt = reinterpret_cast<__half *>(b + offs[i++]);
   p->h = reinterpret_cast<__half *>(b + offs[i++]);
   p->y = reinterpret_cast<__half *>(b + offs[i++]);
-  p->hsmall = reinterpret_cast<float *>(b + offs[i++]);
+  p->hsmall = reinterpret_cast<__half *>(b + offs[i++]);
   p->status = reinterpret_cast<DevStatus *>(b + offs[i++]);
-  p->barrier = reinterpret_cast<uint32_t *>(b + offs[i++]);
+  p->small_sync = reinterpret_cast<uint32_t *>(b + offs[i++]);
   p->x_stage = reinterpret_cast<uint16_t *>(b + offs[i++]);
   p->logits_stage = reinterpret_cast<float *>(b + offs[i++]);
+  p->router_logits = reinterpret_cast<float *>(b + offs[i++]);
   p->out_stage = reinterpret_cast<uint16_t *>(b + offs[i++]);
   err = cudaMemset(p->ws, 0, total);
   if (err == cudaSuccess) err = cudaDeviceSynchronize();
@@ -390,6 +431,40 @@ moe_status moe_forward(moe_plan_t *plan, int T, const void *x_bf16, const float 
   const LayerWeights w = make_weights(packed_w, scales, biases, shared_packed_w, shared_scales, shared_biases);
   return enqueue_layer(plan, T, static_cast<const uint16_t *>(x_bf16), router_logits, w, nullptr,
                        static_cast<uint16_t *>(out_bf16), reinterpret_cast<cudaStream_t>(stream));
+}
+
+moe_status moe_forward_router(moe_plan_t *plan, int T, const void *x_bf16, const void *router_w_bf16,
+                              const uint32_t *packed_w, const void *scales, const void *biases,
+                              const uint32_t *shared_packed_w, const void *shared_scales, const void *shared_biases,
+                              void *out_bf16, moe_stream_t stream) {
+  g_last_error.clear();
+  if (!plan) return fail(MOE_ERR_INVALID_ARG, "plan is NULL");
+  if (T < 0 || T > plan->T_max) return fail(MOE_ERR_INVALID_ARG, "T=%d outside [0, T_max=%d]", T, plan->T_max);
+  if (T == 0) return MOE_OK;
+  if (!x_bf16 || !router_w_bf16 || !out_bf16) return fail(MOE_ERR_INVALID_ARG, "x, router_w and out must not be NULL");
+  if (!aligned16(x_bf16) || !aligned16(router_w_bf16) || !aligned16(out_bf16))
+    return fail(MOE_ERR_INVALID_ARG, "x, router_w and out must be 16-byte aligned");
+  if (x_bf16 == out_bf16) return fail(MOE_ERR_INVALID_ARG, "out must not alias x");
+  moe_status st = check_weights(plan, packed_w, scales, biases, shared_packed_w, shared_scales, shared_biases);
+  if (st != MOE_OK) return st;
+  const LayerWeights w = make_weights(packed_w, scales, biases, shared_packed_w, shared_scales, shared_biases);
+  return enqueue_layer(plan, T, static_cast<const uint16_t *>(x_bf16), nullptr, w, nullptr,
+                       static_cast<uint16_t *>(out_bf16), reinterpret_cast<cudaStream_t>(stream),
+                       static_cast<const uint16_t *>(router_w_bf16));
+}
+
+moe_status moe_router_logits(moe_plan_t *plan, int T, const void *x_bf16, const void *router_w_bf16,
+                             float *logits_out, moe_stream_t stream) {
+  g_last_error.clear();
+  if (!plan) return fail(MOE_ERR_INVALID_ARG, "plan is NULL");
+  if (T < 0 || T > plan->T_max) return fail(MOE_ERR_INVALID_ARG, "T=%d outside [0, T_max=%d]", T, plan->T_max);
+  if (T == 0) return MOE_OK;
+  if (!x_bf16 || !router_w_bf16 || !logits_out)
+    return fail(MOE_ERR_INVALID_ARG, "x, router_w and logits_out must not be NULL");
+  if (!aligned16(x_bf16) || !aligned16(router_w_bf16) || !aligned16(logits_out))
+    return fail(MOE_ERR_INVALID_ARG, "x, router_w and logits_out must be 16-byte aligned");
+  return enqueue_router(plan, T, static_cast<const uint16_t *>(x_bf16), static_cast<const uint16_t *>(router_w_bf16),
+                        logits_out, reinterpret_cast<cudaStream_t>(stream));
 }
 
 moe_status moe_forward_host(moe_plan_t *plan, int T, const void *x_bf16_host, const float *router_logits_host,
@@ -510,9 +585,9 @@ moe_status moe_status_sync(moe_plan_t *plan, moe_stream_t stream) {
   DevStatus h;
   MOE_CUDA(cudaMemcpy(&h, plan->status, sizeof h, cudaMemcpyDeviceToHost), "read status");
   if (h.code == kDevOk) return MOE_OK;
-  // clear the status and the grid barrier so the plan can be used again
+  // clear the status and the small-T counters so the plan can be used again
   MOE_CUDA(cudaMemset(plan->status, 0, sizeof(DevStatus)), "clear status");
-  MOE_CUDA(cudaMemset(plan->barrier, 0, 16), "clear barrier");
+  MOE_CUDA(cudaMemset(plan->small_sync, 0, kSmallTSyncWords * 4), "clear small-T counters");
   MOE_CUDA(cudaDeviceSynchronize(), "synchronize");
   if (h.code == kDevTimeout)
     return fail(MOE_ERR_DEVICE_TIMEOUT, "device wait ran out (site %u, block %u)", h.where, h.detail);

@@ -11,10 +11,19 @@
 namespace moe {
 
 __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
+  pdl_wait();
+  pdl_trigger();
   const int t = blockIdx.x;
   const int H = a.H, k = a.k;
   __shared__ int rows[kMaxTopK + 1];
-  if (threadIdx.x < k) rows[threadIdx.x] = a.inv[static_cast<size_t>(t) * k + threadIdx.x];
+  if (threadIdx.x < k) {
+    int r = a.inv[static_cast<size_t>(t) * k + threadIdx.x];
+    if (a.debug && (r < 0 || r >= a.R)) {  // MOE_FLAG_DEBUG: report and leave the slot out
+      report_error(a.status, kDevBounds, 60, static_cast<uint32_t>(t * k + threadIdx.x));
+      r = -1;
+    }
+    rows[threadIdx.x] = r;
+  }
   if (threadIdx.x == 0) rows[k] = a.R + t;
   __syncthreads();
   const int e2 = 2 * a.xexp[t];
@@ -23,6 +32,7 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
 #pragma unroll
     for (int q = 0; q < 8; ++q) acc[q] = 0.f;
     for (int j = 0; j <= k; ++j) {
+      if (rows[j] < 0) continue;
       const uint4 v = __ldcs(reinterpret_cast<const uint4 *>(a.y + static_cast<size_t>(rows[j]) * H) + c);
       const __half2 *hv = reinterpret_cast<const __half2 *>(&v);
 #pragma unroll
@@ -51,10 +61,9 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
   }
 }
 
-cudaError_t launch_combine(const CombineArgs &a, cudaStream_t s) {
+cudaError_t launch_combine(const CombineArgs &a, cudaStream_t s, bool pdl) {
   if (a.T <= 0) return cudaSuccess;
-  combine_kernel<<<a.T, 256, 0, s>>>(a);
-  return cudaGetLastError();
+  return launch_k(combine_kernel, dim3(a.T), dim3(256), 0, s, pdl, a);
 }
 
 }  // namespace moe

@@ -38,6 +38,18 @@ __device__ __forceinline__ void report_error(DevStatus *st, uint32_t code, uint3
 
 // Budget for every spin-wait: about two seconds of wall clock.
 constexpr unsigned long long kWaitBudgetNs = 2000000000ull;
+// Budget of the waits of a launch that carries the test fault (plan flag
+// MOE_FLAG_TEST_WAIT_TIMEOUT): the wait that cannot succeed gives up quickly.
+constexpr unsigned long long kTestWaitBudgetNs = 2000000ull;
+
+// Programmatic dependent launch. Every kernel of the grouped path runs its
+// independent prologue (barrier set-up, tensor-memory allocation, descriptor
+// prefetch), then pdl_wait() -- which returns once the kernels it depends on
+// have completed and their writes are visible (at once when it was launched
+// in plain stream order) -- before its first global-memory access, and then
+// pdl_trigger() so the next kernel on the stream may be scheduled early.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 __device__ __forceinline__ unsigned long long global_ns() {
   unsigned long long t;
@@ -95,7 +107,9 @@ namespace moe {
 // each, by one fp16 FMA), returned in the K-permuted operand order.
 // The nibble is placed in the mantissa of an fp16 with a fixed exponent
 // (1024 + q for bits 0..3, 64 + q for bits 4..7) and the offset subtracted
-// exactly; this is the usual bit-trick int4 -> fp16 conversion.
+// exactly: the magic-number int4 -> fp16 conversion published with the MARLIN
+// mixed-precision kernels (Frantar et al., arXiv:2408.11743), which also
+// yields the pair order (0,4), (1,5), (2,6), (3,7) used for the operands.
 __device__ __forceinline__ uint4 dequant_word(uint32_t w, __half2 s2, __half2 b2) {
   const uint32_t hi = w >> 8;
   const uint32_t a0 = (w & 0x000F000Fu) | 0x64006400u;   // {1024+n0, 1024+n4}

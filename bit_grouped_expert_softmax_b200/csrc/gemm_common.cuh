@@ -44,6 +44,34 @@ __device__ __forceinline__ void drain_stages(uint64_t *full, uint32_t issued, ui
   }
 }
 
+// Whether a work item lies inside the buffers it addresses: its expert, its
+// 128-row weight block and its activation rows (routed rows in [0, R), the
+// shared expert's rows in [R, R + T)); every TMA coordinate of the item
+// derives from these. dn: the down GEMM (weight rows H) or gate/up (I or Is).
+__device__ __forceinline__ bool item_in_range(const GemmArgs &a, const WorkItem &wi, bool dn) {
+  if (wi.group < 0 || wi.group > a.E) return false;
+  const bool sh = wi.group == a.E;
+  const int mrows = dn ? a.H : (sh ? a.Is : a.I);
+  if (wi.mblk < 0 || wi.mblk >= mrows / kTileM) return false;
+  if (wi.nrows < 1 || wi.nrows > kTileN || wi.row0 < 0) return false;
+  const int64_t end = static_cast<int64_t>(wi.row0) + wi.nrows;
+  if (sh) return wi.row0 >= a.R && end <= static_cast<int64_t>(a.R) + a.T;
+  return end <= a.R;
+}
+
+// The first work item at or after `it` (stepping by the grid) that this CTA
+// processes. Without MOE_FLAG_DEBUG that is `it`; with it, items out of range
+// are skipped by every warp role alike (so the pipelines stay in step), and
+// the role that passes report = true records each one in the status word.
+__device__ __forceinline__ int next_item(const GemmArgs &a, int it, int nitems, bool dn, bool report) {
+  if (!a.debug) return it;
+  while (it < nitems && !item_in_range(a, a.items[it], dn)) {
+    if (report) report_error(a.status, kDevBounds, dn ? 150u : 250u, static_cast<uint32_t>(it));
+    it += gridDim.x;
+  }
+  return it;
+}
+
 // 2^e as a float for |e| <= 126, built from its exponent bits
 __device__ __forceinline__ float pow2i(int e) { return __int_as_float((127 + e) << 23); }
 
@@ -88,6 +116,19 @@ __device__ __forceinline__ void dequant4(uint4 v, __half2 s2, __half2 b2, uint32
     d[4 * cw + 2] = o.z;
     d[4 * cw + 3] = o.w;
   }
+}
+
+// Dequantise two packed words (16 weights of one row) into 8 fp16 pairs.
+__device__ __forceinline__ void dequant2(uint32_t w0, uint32_t w1, __half2 s2, __half2 b2, uint32_t (&d)[8]) {
+  const uint4 o0 = dequant_word(w0, s2, b2), o1 = dequant_word(w1, s2, b2);
+  d[0] = o0.x;
+  d[1] = o0.y;
+  d[2] = o0.z;
+  d[3] = o0.w;
+  d[4] = o1.x;
+  d[5] = o1.y;
+  d[6] = o1.z;
+  d[7] = o1.w;
 }
 
 // Dequantise eight packed words (one row's K-block of 64 weights) into 32 fp16 pairs.

@@ -131,6 +131,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_down_kernel(const GemmArgs a
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // the prologue above touched no global memory; the routing results, the
+  // activation rows and the work list come from the kernels before this one
+  pdl_wait();
+  pdl_trigger();
 
   const int nitems = min(*a.item_count, a.max_items);
   const int H = a.H;
@@ -141,7 +145,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_down_kernel(const GemmArgs a
       int s = 0;
       uint32_t ph = 0, issued = 0, issued_ph = 0;
       bool ok = true;
-      for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
+      for (int it = next_item(a, blockIdx.x, nitems, true, true); it < nitems && ok;
+           it = next_item(a, it + gridDim.x, nitems, true, true)) {
         const WorkItem wi = a.items[it];
         const bool sh = wi.group == a.E;
         const int K = sh ? a.Is : a.I;
@@ -171,7 +176,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_down_kernel(const GemmArgs a
       int s = 0;
       uint32_t ph = 0, issued = 0, issued_ph = 0;
       bool ok = true;
-      for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
+      for (int it = next_item(a, blockIdx.x, nitems, true, false); it < nitems && ok;
+           it = next_item(a, it + gridDim.x, nitems, true, false)) {
         const WorkItem wi = a.items[it];
         const bool sh = wi.group == a.E;
         const int K = sh ? a.Is : a.I;
@@ -205,7 +211,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_down_kernel(const GemmArgs a
     uint32_t phb = 0, pha = 0;
     bool ok = true;
     int li = 0;
-    for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x, ++li) {
+    for (int it = next_item(a, blockIdx.x, nitems, true, false); it < nitems && ok;
+         it = next_item(a, it + gridDim.x, nitems, true, false), ++li) {
       const WorkItem wi = a.items[it];
       const int K = wi.group == a.E ? a.Is : a.I;
       const int st = li % kAccStages;
@@ -265,18 +272,27 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_down_kernel(const GemmArgs a
     // this warp's 32 output columns of the tile's rows, staged as [row][32] fp16
     __half *stg = reinterpret_cast<__half *>(smem + kOffStg + (warp - kEpiWarp0) * kStgBytes);
     int li = 0;
-    for (int it = blockIdx.x; it < nitems; it += gridDim.x, ++li) {
+    for (int it = next_item(a, blockIdx.x, nitems, true, false); it < nitems;
+         it = next_item(a, it + gridDim.x, nitems, true, false), ++li) {
       const WorkItem wi = a.items[it];
       const int st = li % kAccStages;
       const uint32_t acc_ph = (li / kAccStages) & 1;
+      // routing weight of each row, lane l of chunk c holding row 32c + l,
+      // loaded before the accumulators are ready
+      static_assert(kN / 32 == 4, "four 32-row chunks per tile");
+      float w_l[kN / 32];
+#pragma unroll
+      for (int c = 0; c < kN / 32; ++c) {
+        const int jl = 32 * c + lane;
+        w_l[c] = jl < wi.nrows ? a.row_w[wi.row0 + jl] : 0.f;
+      }
       if (!warp_wait(&acc_full[st], acc_ph, abort, a.status, 120)) break;
       tc_fence_after();
       const uint32_t tq = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + st * kN;
       __half *obase = a.y + static_cast<int64_t>(wi.row0) * H + wi.mblk * kTileM + q * 32;
       for (int c0 = 0; c0 < wi.nrows; c0 += 32) {
-        // routing weight of each row, one row per lane, broadcast by shuffles
-        const int jl = c0 + lane;
-        const float wl = jl < wi.nrows ? a.row_w[wi.row0 + jl] : 0.f;
+        const int c = c0 >> 5;
+        const float wl = c == 0 ? w_l[0] : c == 1 ? w_l[1] : c == 2 ? w_l[2] : w_l[3];
         uint32_t r0[32];
         tmem_ld_32x32b_x32(tq + c0, r0);
         tmem_ld_wait();
@@ -317,11 +333,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_down_kernel(const GemmArgs a
     // first stage of the next item is fetched during the last stage of this one
     SbRow row{};
     uint2 s_cur{}, b_cur{}, s_nxt{}, b_nxt{};
-    if (blockIdx.x < nitems) {
-      row = sb_row_dn(a, a.items[blockIdx.x], r);
+    const int first = next_item(a, blockIdx.x, nitems, true, false);
+    if (first < nitems) {
+      row = sb_row_dn(a, a.items[first], r);
       load_sb4(row, 0, s_nxt, b_nxt);
     }
-    for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
+    for (int it = first; it < nitems && ok; it = next_item(a, it + gridDim.x, nitems, true, false)) {
       const int nkb = row.K / kTileK;
       SbRow next_row = row;
       for (int kb = 0; kb < nkb; ++kb) {
@@ -331,8 +348,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_down_kernel(const GemmArgs a
           b_cur = b_nxt;
           if (kb + kSuperK < nkb) {
             load_sb4(row, kb + kSuperK, s_nxt, b_nxt);
-          } else if (it + static_cast<int>(gridDim.x) < nitems) {
-            next_row = sb_row_dn(a, a.items[it + gridDim.x], r);
+          } else if (const int nx = next_item(a, it + gridDim.x, nitems, true, false); nx < nitems) {
+            next_row = sb_row_dn(a, a.items[nx], r);
             load_sb4(next_row, 0, s_nxt, b_nxt);
           }
         }
@@ -384,7 +401,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_down_kernel(const GemmArgs a
 
 }  // namespace
 
-cudaError_t launch_gemm_down(const GemmArgs &a, int num_sms, cudaStream_t s) {
+cudaError_t launch_gemm_down(const GemmArgs &a, int num_sms, cudaStream_t s, bool pdl) {
   if (a.max_items <= 0) return cudaSuccess;
   TmaMaps maps;
   const int H = a.H;
@@ -401,8 +418,7 @@ cudaError_t launch_gemm_down(const GemmArgs &a, int num_sms, cudaStream_t s) {
   const cudaError_t e = ensure_smem_limit(gemm_down_kernel, kSmem, smem_set);
   if (e != cudaSuccess) return e;
   const int grid = std::max(1, std::min(num_sms, a.max_items));
-  gemm_down_kernel<<<grid, kThreads, kSmem, s>>>(a, maps);
-  return cudaGetLastError();
+  return launch_k(gemm_down_kernel, dim3(grid), dim3(kThreads), kSmem, s, pdl, a, maps);
 }
 
 }  // namespace moe

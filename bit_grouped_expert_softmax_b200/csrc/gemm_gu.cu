@@ -136,6 +136,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_gate_up_kernel(const GemmArg
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // the prologue above touched no global memory; the routing results, the
+  // activation rows and the work list come from the kernels before this one
+  pdl_wait();
+  pdl_trigger();
 
   const int nitems = min(*a.item_count, a.max_items);
   const int H = a.H;
@@ -147,7 +151,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_gate_up_kernel(const GemmArg
       int s = 0;
       uint32_t ph = 0, issued = 0, issued_ph = 0;
       bool ok = true;
-      for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
+      for (int it = next_item(a, blockIdx.x, nitems, false, true); it < nitems && ok;
+           it = next_item(a, it + gridDim.x, nitems, false, true)) {
         const WorkItem wi = a.items[it];
         const bool sh = wi.group == a.E;
         const int base = sh ? 0 : wi.group * 3 * a.I;  // rows of H/8 words
@@ -179,7 +184,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_gate_up_kernel(const GemmArg
       int s = 0;
       uint32_t ph = 0, issued = 0, issued_ph = 0;
       bool ok = true;
-      for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
+      for (int it = next_item(a, blockIdx.x, nitems, false, false); it < nitems && ok;
+           it = next_item(a, it + gridDim.x, nitems, false, false)) {
         const WorkItem wi = a.items[it];
         const int nb = (wi.nrows + kBRows - 1) / kBRows;
         for (int ks = 0; ks < nkb / kStageK; ++ks) {
@@ -209,7 +215,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_gate_up_kernel(const GemmArg
     uint32_t phb = 0, pha = 0;
     bool ok = true;
     int li = 0;
-    for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x, ++li) {
+    for (int it = next_item(a, blockIdx.x, nitems, false, false); it < nitems && ok;
+         it = next_item(a, it + gridDim.x, nitems, false, false), ++li) {
       const WorkItem wi = a.items[it];
       if (!warp_wait(acc_empty, (li & 1) ^ 1u, abort, a.status, 210)) break;
       tc_fence_after();
@@ -332,11 +339,12 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_gate_up_kernel(const GemmArg
     // first stage of the next item is fetched during the last stage of this one
     SbRow row{};
     uint2 s_cur{}, b_cur{}, s_nxt{}, b_nxt{};
-    if (blockIdx.x < nitems) {
-      row = sb_row_gu(a, a.items[blockIdx.x], m, r);
+    const int first = next_item(a, blockIdx.x, nitems, false, false);
+    if (first < nitems) {
+      row = sb_row_gu(a, a.items[first], m, r);
       load_sb4(row, 0, s_nxt, b_nxt);
     }
-    for (int it = blockIdx.x; it < nitems && ok; it += gridDim.x) {
+    for (int it = first; it < nitems && ok; it = next_item(a, it + gridDim.x, nitems, false, false)) {
       SbRow next_row = row;
       for (int kb = 0; kb < nkb; ++kb) {
         const int j = kb % kSuperK;
@@ -345,14 +353,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_gate_up_kernel(const GemmArg
           b_cur = b_nxt;
           if (kb + kSuperK < nkb) {
             load_sb4(row, kb + kSuperK, s_nxt, b_nxt);
-          } else if (it + static_cast<int>(gridDim.x) < nitems) {
-            next_row = sb_row_gu(a, a.items[it + gridDim.x], m, r);
+          } else if (const int nx = next_item(a, it + gridDim.x, nitems, false, false); nx < nitems) {
+            next_row = sb_row_gu(a, a.items[nx], m, r);
             load_sb4(next_row, 0, s_nxt, b_nxt);
           }
-        }
-        if (!warp_wait(&a_empty[sa], pha ^ 1u, abort, a.status, 231)) {
-          ok = false;
-          break;
         }
         const __half2 s2 = bf16_to_half2_bcast(pick_bf16(s_cur, j));
         const __half2 b2 = bf16_to_half2_bcast(pick_bf16(b_cur, j));
@@ -373,10 +377,23 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_gate_up_kernel(const GemmArg
             php ^= 1u;
           }
         }
-        uint32_t dq[32];
-        dequant8(v0, v1, s2, b2, dq);
-        tmem_st_32x32b_x32(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + kACol0 + sa * kAStageCols + m * 32,
-                           dq);
+        // four quarters of the K-block: each quarter's store to tensor memory
+        // is in flight while the next quarter is dequantised; one wait at the
+        // end. The first quarter is computed before the stage is known free.
+        const uint32_t ta = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + kACol0 + sa * kAStageCols + m * 32;
+        uint32_t d8[8];
+        dequant2(v0.x, v0.y, s2, b2, d8);
+        if (!warp_wait(&a_empty[sa], pha ^ 1u, abort, a.status, 231)) {
+          ok = false;
+          break;
+        }
+        tmem_st_32x32b_x8(ta, d8);
+        dequant2(v0.z, v0.w, s2, b2, d8);
+        tmem_st_32x32b_x8(ta + 8, d8);
+        dequant2(v1.x, v1.y, s2, b2, d8);
+        tmem_st_32x32b_x8(ta + 16, d8);
+        dequant2(v1.z, v1.w, s2, b2, d8);
+        tmem_st_32x32b_x8(ta + 24, d8);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
@@ -400,7 +417,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_gate_up_kernel(const GemmArg
 
 }  // namespace
 
-cudaError_t launch_gemm_gate_up(const GemmArgs &a, int num_sms, cudaStream_t s) {
+cudaError_t launch_gemm_gate_up(const GemmArgs &a, int num_sms, cudaStream_t s, bool pdl) {
   if (a.max_items <= 0) return cudaSuccess;
   TmaMaps maps;
   const int H = a.H;
@@ -416,8 +433,7 @@ cudaError_t launch_gemm_gate_up(const GemmArgs &a, int num_sms, cudaStream_t s) 
   const cudaError_t e = ensure_smem_limit(gemm_gate_up_kernel, kSmem, smem_set);
   if (e != cudaSuccess) return e;
   const int grid = std::max(1, std::min(num_sms, a.max_items));
-  gemm_gate_up_kernel<<<grid, kThreads, kSmem, s>>>(a, maps);
-  return cudaGetLastError();
+  return launch_k(gemm_gate_up_kernel, dim3(grid), dim3(kThreads), kSmem, s, pdl, a, maps);
 }
 
 }  // namespace moe

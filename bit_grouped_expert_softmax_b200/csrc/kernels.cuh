@@ -1,6 +1,8 @@
 // kernels.cuh -- argument blocks and launch declarations of the MoE kernels.
 #pragma once
 
+#include <utility>
+
 #include "common.cuh"
 
 namespace moe {
@@ -20,13 +22,15 @@ struct RouteScanArgs {
   WorkItem *dn_items;   // down work list
   int max_dn;
   int32_t *item_counts; // [0] gate/up items, [1] down items
+  int32_t *done;        // blocks finished (zero between launches)
   DevStatus *status;
 };
 
 struct RouteScatterArgs {
   int T, E, k, H;
   const int32_t *ids;         // [T*k]
-  int32_t *chunk_base;        // [nchunk][E] bases in; zeroed on the way out
+  int32_t *chunk_base;        // [nchunk][E] per-chunk prefixes in; zeroed on the way out
+  const int32_t *offsets;     // [E+1] first row of each expert
   int32_t *perm;              // [T*k]
   int32_t *inv;               // [T*k]
   const uint16_t *x;          // [T, H] bf16, or null (routing only)
@@ -68,6 +72,7 @@ struct GemmArgs {
   int64_t h_rows;           // routed h rows allocated
   int64_t hs_rows;          // shared h rows allocated
   DevStatus *status;
+  int debug;                // MOE_FLAG_DEBUG: range-check every work item, skip and report bad ones
 };
 
 struct CombineArgs {
@@ -77,17 +82,37 @@ struct CombineArgs {
   const int32_t *xexp;       // [T]
   const uint16_t *residual;  // [T, H] bf16 or null
   uint16_t *out;             // [T, H] bf16 (may alias residual)
+  DevStatus *status;
+  int debug;                 // MOE_FLAG_DEBUG: range-check every inverse-permutation entry
 };
+
+// Distinct experts one small-T launch can use: the shared one plus T*k routed.
+constexpr int kSmallTMaxU = kSmallT * kMaxTopK + 1;
+// Synchronisation words of the small-T kernel: one readiness counter per used
+// expert, the exit counter, then the count of CTAs whose router scores are
+// published. They must be zero before a launch; each launch leaves them zero.
+constexpr int kSmallTSyncWords = kSmallTMaxU + 2;
 
 struct SmallTArgs {
   int T, E, k, H, I, Is;
   const uint16_t *x;        // [T, H] bf16
-  const float *logits;      // [T, E]
+  const float *logits;      // [T, E]; written by the kernel itself when router_w is set
+  const uint16_t *router_w; // [E, H] bf16 router weight, or null (logits given)
   LayerWeights w;
-  float *hbuf;              // [(T*k+1), T, max(I,Is)] fp32 scratch
-  uint32_t *barrier;        // grid barrier {count, generation}
+  __half *hbuf;             // [8][k+1][max(I,Is)] fp16 scratch: SwiGLU outputs by token and slot
+  uint32_t *sync;           // [kSmallTSyncWords] readiness and exit counters (zero between launches)
   const uint16_t *residual; // [T, H] or null
   uint16_t *out;            // [T, H]
+  DevStatus *status;
+  unsigned long long wait_ns;  // budget of every bounded wait
+  int test_fault;           // testing only: row block 0 of the shared expert does not publish its h
+};
+
+struct RouterArgs {
+  int T, E, H;
+  const uint16_t *x;        // [T, H] bf16
+  const uint16_t *w;        // [E, H] bf16 router weight
+  float *logits;            // [T, E] float32 scores
   DevStatus *status;
 };
 
@@ -98,10 +123,29 @@ __global__ void route_scan_kernel(RouteScanArgs a);
 __global__ void route_scatter_kernel(RouteScatterArgs a);
 __global__ void gather_kernel(RouteScatterArgs a);
 
+// Launch with the programmatic-stream-serialisation attribute when pdl is set
+// (the kernel must call pdl_wait() before its first global-memory access).
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_k(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, bool pdl,
+                            Args &&...args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 // host-side launchers (each returns the launch's cudaError_t)
-cudaError_t launch_gemm_gate_up(const GemmArgs &a, int num_sms, cudaStream_t s);
-cudaError_t launch_gemm_down(const GemmArgs &a, int num_sms, cudaStream_t s);
-cudaError_t launch_combine(const CombineArgs &a, cudaStream_t s);
+cudaError_t launch_gemm_gate_up(const GemmArgs &a, int num_sms, cudaStream_t s, bool pdl);
+cudaError_t launch_gemm_down(const GemmArgs &a, int num_sms, cudaStream_t s, bool pdl);
+cudaError_t launch_combine(const CombineArgs &a, cudaStream_t s, bool pdl);
+cudaError_t launch_router(const RouterArgs &a, cudaStream_t s, bool pdl);
 cudaError_t launch_small_t(const SmallTArgs &a, int num_sms, cudaStream_t s);
 int small_t_grid(int num_sms);
 // whether the fused small-T kernel can run this layer (shared memory, grid)

@@ -7,8 +7,10 @@
 // Four kernels:
 //   route_topk_kernel    softmax over E, warp top-k, renormalised weights,
 //                        per-chunk expert histogram
-//   route_scan_kernel    per-expert totals, exclusive scan (offsets), per-chunk
-//                        bases, and the grouped-GEMM work lists (block map)
+//   route_scan_kernel    per-expert totals and per-chunk prefixes (one warp per
+//                        expert), then, in the last block to finish, the
+//                        exclusive scan (offsets) and the grouped-GEMM work
+//                        lists (block map)
 //   route_scatter_kernel stable permutation (experts ascending, tokens ascending
 //                        within an expert) and its inverse
 //   gather_kernel        each token's row, fp16 scaled by a power of two, copied
@@ -27,6 +29,8 @@ __global__ void __launch_bounds__(256) route_topk_kernel(int T, int E, int k,
                                                          int32_t *__restrict__ chunk_cnt) {
   // one warp per token; the per-chunk expert histogram is built with integer
   // atomics (order-independent) into chunk_cnt, which starts zeroed
+  pdl_wait();
+  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * (blockDim.x >> 5) + warp;
   if (t >= T) return;
@@ -40,39 +44,56 @@ __global__ void __launch_bounds__(256) route_topk_kernel(int T, int E, int k,
   }
 }
 
-// Single block. Turns per-chunk counts into per-chunk bases (in place), writes
-// offsets[0..E] and the two work lists.
-__global__ void __launch_bounds__(1024) route_scan_kernel(RouteScanArgs a) {
-  __shared__ int tot[kMaxExperts + 1];
+// One warp per expert (8 per block). Each warp turns its expert's column of
+// per-chunk counts into exclusive prefix sums over the chunks (in place: the
+// rows each chunk's first entry lands at, relative to the expert's first row)
+// and leaves the expert's total in offsets[e]. The last block to finish
+// (counted in *done) scans the totals into offsets[0..E] and writes the two
+// work lists (block map), then resets *done for the next launch.
+__global__ void __launch_bounds__(256) route_scan_kernel(RouteScanArgs a) {
   __shared__ int off[kMaxExperts + 2];
   __shared__ int gu_off[kMaxExperts + 2];
   __shared__ int dn_off[kMaxExperts + 2];
-  __shared__ int warp_tot[3][32];
-  __shared__ int part[4][kMaxExperts];
+  __shared__ int tot[kMaxExperts + 1];
+  __shared__ int totals3[3];
+  __shared__ int is_last;
+  pdl_wait();
+  pdl_trigger();
   const int E = a.E;
-  const int G = E + 1;  // routed experts plus the shared one
-  // each expert's column of per-chunk counts is split into four slices; the
-  // loads of a slice are issued in batches so they overlap
-  const int nq = (a.nchunk + 3) / 4;
-  const int e_t = threadIdx.x >> 2, q_t = threadIdx.x & 3;
-  const int c_lo = q_t * nq, c_hi = min(a.nchunk, c_lo + nq);
-  if (e_t < E) {
-    int sum = 0;
-    for (int c = c_lo; c < c_hi; c += 8) {
-      int v[8];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int e = blockIdx.x * 8 + warp;
+  if (e < E) {
+    int run = 0;
+    for (int c0 = 0; c0 < a.nchunk; c0 += 128) {
+      int v[4];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) v[u] = (c + u < c_hi) ? __ldcg(a.chunk_cnt + static_cast<size_t>(c + u) * E + e_t) : 0;
+      for (int u = 0; u < 4; ++u) {  // four loads in flight per lane
+        const int c = c0 + 32 * u + lane;
+        v[u] = c < a.nchunk ? __ldcg(a.chunk_cnt + static_cast<size_t>(c) * E + e) : 0;
+      }
 #pragma unroll
-      for (int u = 0; u < 8; ++u) sum += v[u];
+      for (int u = 0; u < 4; ++u) {
+        const int c = c0 + 32 * u + lane;
+        const int incl = warp_incl_scan(v[u]);
+        if (c < a.nchunk) a.chunk_cnt[static_cast<size_t>(c) * E + e] = run + incl - v[u];
+        run += __shfl_sync(0xffffffffu, incl, 31);
+      }
     }
-    part[q_t][e_t] = sum;
+    if (lane == 0) a.offsets[e] = run;  // the expert's total until the last block scans them
+  }
+  __threadfence();  // this thread's prefixes and total are visible before the block counts itself done
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    is_last = atomicAdd(a.done, 1) == static_cast<int>(gridDim.x) - 1;
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < E; e += blockDim.x) tot[e] = part[0][e] + part[1][e] + part[2][e] + part[3][e];
+  if (!is_last) return;
+  __threadfence();
+  for (int g = threadIdx.x; g < E; g += blockDim.x) tot[g] = __ldcg(a.offsets + g);
   __syncthreads();
+  const int G = E + 1;  // routed experts plus the shared one
   // exclusive scans over the groups, done by warp 0 with 9 values per lane (G <= 257)
-  if (threadIdx.x < 32) {
-    const int lane = threadIdx.x;
+  if (warp == 0) {
     constexpr int PER = (kMaxExperts + 1 + 31) / 32;
     int cnt[PER], gu[PER], dn[PER];
     int sc = 0, sg = 0, sd = 0;
@@ -107,41 +128,25 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(RouteScanArgs a) {
       bd += dn[i];
     }
     if (lane == 31) {
-      warp_tot[0][0] = ic;
-      warp_tot[1][0] = ig;
-      warp_tot[2][0] = id;
+      totals3[0] = ic;
+      totals3[1] = ig;
+      totals3[2] = id;
     }
   }
   __syncthreads();
-  for (int e = threadIdx.x; e <= E; e += blockDim.x) a.offsets[e] = (e < E) ? off[e] : a.T * a.k;
-  // per-chunk counts become absolute row positions of each chunk's first entry
-  if (e_t < E) {
-    int base = off[e_t];
-    for (int q = 0; q < q_t; ++q) base += part[q][e_t];
-    for (int c = c_lo; c < c_hi; c += 8) {
-      int v[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) v[u] = (c + u < c_hi) ? __ldcg(a.chunk_cnt + static_cast<size_t>(c + u) * E + e_t) : 0;
-#pragma unroll
-      for (int u = 0; u < 8; ++u)
-        if (c + u < c_hi) {
-          a.chunk_cnt[static_cast<size_t>(c + u) * E + e_t] = base;
-          base += v[u];
-        }
-    }
-  }
+  for (int g = threadIdx.x; g <= E; g += blockDim.x) a.offsets[g] = (g < E) ? off[g] : a.T * a.k;
   // work lists: group g's tiles are (n-tile, m-block) with the m-block fastest,
   // so neighbouring CTAs share the activation tile of one n-tile
   const int R = a.T * a.k;
-  const int gu_total = warp_tot[1][0], dn_total = warp_tot[2][0];
+  const int gu_total = totals3[1], dn_total = totals3[2];
   if (threadIdx.x == 0) {
     if (gu_total > a.max_gu || dn_total > a.max_dn)
       report_error(a.status, kDevBounds, 10, static_cast<uint32_t>(max(gu_total, dn_total)));
     a.item_counts[0] = min(gu_total, a.max_gu);
     a.item_counts[1] = min(dn_total, a.max_dn);
+    *a.done = 0;  // ready for the next launch (the kernel boundary orders it)
   }
-  for (int g = threadIdx.x >> 5; g < G; g += blockDim.x >> 5) {
-    const int lane = threadIdx.x & 31;
+  for (int g = warp; g < G; g += blockDim.x >> 5) {
     const int n = (g < E) ? tot[g] : a.T;
     const int row0 = (g < E) ? off[g] : R;
     const int ntg = (n + kGuTileN - 1) / kGuTileN, ntile = (n + kTileN - 1) / kTileN;
@@ -163,9 +168,13 @@ __global__ void __launch_bounds__(1024) route_scan_kernel(RouteScanArgs a) {
 // bases is reset to zero afterwards, ready for the next routing's histogram.
 __global__ void __launch_bounds__(256) route_scatter_kernel(RouteScatterArgs a) {
   __shared__ int cnt[kMaxExperts];
+  pdl_wait();
+  pdl_trigger();
   const int chunk = blockIdx.x, E = a.E, k = a.k, T = a.T;
   int32_t *row = a.chunk_base + static_cast<size_t>(chunk) * E;
-  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = __ldcg(row + e);
+  // the chunk's first row of each expert: the expert's offset plus the
+  // entries of earlier chunks (the scan's per-chunk prefix)
+  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = __ldcg(row + e) + __ldcg(a.offsets + e);
   __syncthreads();
   for (int e = threadIdx.x; e < E; e += blockDim.x) row[e] = 0;
   const int t0 = chunk * kRouteChunk, t1 = min(T, t0 + kRouteChunk);
@@ -204,6 +213,8 @@ __global__ void __launch_bounds__(256) route_scatter_kernel(RouteScatterArgs a) 
 // the token's k routed rows (positions from the scatter) and its shared-expert
 // row R + t.
 __global__ void __launch_bounds__(256) gather_kernel(RouteScatterArgs a) {
+  pdl_wait();
+  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * (blockDim.x >> 5) + warp;
   if (t >= a.T) return;

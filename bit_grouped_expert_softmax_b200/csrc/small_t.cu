@@ -2,24 +2,36 @@
 //
 // Batch-1 decode has almost no weight reuse, so memory bandwidth sets the
 // ceiling (aioga.com record of the Lily report, article body paragraph 6).
-// One persistent cooperative kernel, one CTA per SM, does the whole layer so
-// that every weight byte it needs is requested as early as possible:
+// One persistent cooperative kernel, one CTA per SM, does the whole layer and
+// requests every weight byte it needs as early as the data dependences allow:
 //
-//   phase 0  every CTA routes the (<= 8) tokens itself (same result in every
-//            CTA), lists the distinct experts used, stages the tokens as fp16
-//            (scaled by a power of two per token) in the operand order below,
-//            and requests -- with bulk asynchronous copies into shared memory --
-//            the gate/up row blocks and the down-projection rows it will need;
-//            the shared expert's first block is requested before routing ends
-//   phase 1  gate/up: each 16-row block of an expert is split along K over
-//            several warps; tensor-core mma.sync m16n8k16 with A = dequantised
-//            weights (fp16 q*scale+bias, as in the grouped GEMM) and B = the
-//            tokens (N = 8 covers every token at once); partial sums reduced in
-//            a fixed order, then h = silu(gate) * up goes to a small scratch
-//   barrier  bounded grid barrier (the launch is cooperative)
-//   phase 2  down: each CTA owns 16 output features; its warps take the used
-//            experts, weighting each token's result by its routing weight; the
-//            warps' results are summed in a fixed order and rounded once
+//   entry    the shared expert needs no routing: each CTA requests, with bulk
+//            asynchronous copies into shared memory, its shared-expert gate/up
+//            row block and the shared expert's down rows of its output slice
+//            before it looks at a logit
+//   routing  every CTA routes the (<= 8) tokens itself (same result in every
+//            CTA) with all its warps: each warp takes the top k of one 32-expert
+//            slice of one token, then one warp per token merges the slices'
+//            candidates; the distinct experts are listed and their gate/up row
+//            blocks and down rows requested at once, from several warps
+//   gate/up  each 16-row block of an expert is split along K over several
+//            warps; tensor-core mma.sync m16n8k16 with A = dequantised weights
+//            (fp16 q*scale+bias, as in the grouped GEMM) and B = the tokens
+//            (N = 8 covers every token at once); partial sums reduced in a fixed
+//            order, h = silu(gate) * up written to a small scratch, and the
+//            expert's readiness counter incremented (release)
+//   down     each CTA owns 16 output features; warp w takes the used experts
+//            u = w, w + 16, ...; it waits (bounded, acquire) until every row
+//            block of expert u has published its h, then multiplies that h by
+//            the down rows already in shared memory and weights each token's
+//            result by its routing weight; the warps' results are summed in a
+//            fixed order and rounded once
+//   exit     the last CTA to leave resets the readiness counters for the next
+//            launch on the stream; a CTA that gave up on a wait first waits for
+//            its own copies still in flight
+//
+// There is no grid-wide barrier: an expert's down product starts as soon as
+// that expert's h is complete, while other experts' gate/up blocks finish.
 //
 // Operand order along K: packed word W holds elements 8W..8W+7; the fp16
 // operands store them at positions 8W + s in the pair order (0,4),(1,5),(2,6),
@@ -29,6 +41,7 @@
 // product.
 #include <algorithm>
 
+#include "gemm_common.cuh"
 #include "kernels.cuh"
 #include "sm100.cuh"
 #include "topk.cuh"
@@ -43,18 +56,23 @@ constexpr int kSTWarps = 16;
 constexpr int kSTThreads = kSTWarps * 32;
 constexpr int kRowBlock = 16;  // weight rows per mma tile
 constexpr int kXPad = 32;      // fp16 padding per staged token row (bank spread)
-constexpr int kMaxU = kSmallT * kMaxTopK + 1;
+constexpr int kSlices = kMaxExperts / 32;  // 32-expert slices of a token's logits
+constexpr int kCandPerToken = kSlices * kMaxTopK;  // routing candidates of one token, at most
+static_assert(kSmallTMaxU == kSmallT * kMaxTopK + 1, "one shared plus at most T*k routed experts");
+constexpr int kMaxU = kSmallTMaxU;
 
 struct SmallTShared {
   int ids[kSmallT][kMaxTopK];
+  uint32_t wkey[kSmallT][kMaxTopK];     // order keys of the chosen experts' logits
   float wt[kSmallT][kMaxTopK];
   int xexp[kSmallT];                   // max |x| bits, then the token's exponent
   uint32_t bitmap[kMaxExperts / 32];   // experts used by any token
-  int ulist[kMaxU];                    // distinct experts, ascending, then the shared one (E)
+  int ulist[kMaxU];                    // [0] the shared expert (E), then the distinct experts ascending
   uint32_t umask[kMaxU];               // tokens routed to each
   int8_t uslot[kMaxU][kSmallT];        // slot j of expert u in token t (-1: none; k: shared)
+  int b_iss[4];                        // copies issued into each phase-1 stage
+  int d_iss[kMaxU];                    // copies issued into each phase-2 stage
   int nU;
-  int ok;
   int abort;
 };
 
@@ -65,6 +83,8 @@ struct StLayout {
   size_t x_off, red_off, b_off, d_off, bar_off, bytes;
   size_t b_stage, d_stage;
 };
+
+constexpr size_t kStBudget = 220 * 1024;
 
 __host__ __device__ inline StLayout st_layout(int H, int I, int Is, int T, int k) {
   StLayout L;
@@ -80,19 +100,18 @@ __host__ __device__ inline StLayout st_layout(int H, int I, int Is, int T, int k
   L.x_off = 0;
   const size_t x_bytes = static_cast<size_t>(kSmallT) * (H + kXPad) * 2;
   L.red_off = (x_bytes + 127) / 128 * 128;
+  // partial sums of the K slices; during routing, the top-k candidates
   const size_t red_bytes = static_cast<size_t>(kSTThreads) * 8 * 4;
   L.b_off = L.red_off + red_bytes;
-  const size_t budget = 220 * 1024;
-  const size_t h_bytes = static_cast<size_t>(T) * (k + 1) * L.Imax * 2;  // phase-2 copy of h (in the B ring)
   // phase-1 ring: the most stages (up to 4) that still leave the down ring one
-  // stage per used expert (or at least 8); the B ring must also hold h later
+  // stage per used expert (or at least 8)
   const int want_d = T * k + 1;
   L.nb = 0;
   L.nd = 0;
   for (int nb = 4; nb >= 2; --nb) {
     const size_t used = L.b_off + nb * L.b_stage + 512;
-    if (used >= budget || nb * L.b_stage < h_bytes) continue;
-    int nd = static_cast<int>((budget - used) / L.d_stage);
+    if (used >= kStBudget) continue;
+    int nd = static_cast<int>((kStBudget - used) / L.d_stage);
     nd = nd < want_d ? nd : want_d;
     if (nd >= (want_d < 8 ? want_d : 8) || nb == 2) {
       L.nb = nb;
@@ -108,16 +127,53 @@ __host__ __device__ inline StLayout st_layout(int H, int I, int Is, int T, int k
 
 // Bounded wait on an mbarrier phase; on timeout or abort returns false.
 __device__ __forceinline__ bool st_wait(uint64_t *bar, uint32_t parity, volatile int *abort, DevStatus *st,
-                                        uint32_t site) {
+                                        uint32_t site, unsigned long long budget) {
   if (mbar_try_wait(bar, parity)) return true;
   const unsigned long long t0 = global_ns();
   while (true) {
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
-    if (global_ns() - t0 > kWaitBudgetNs) {
+    if (global_ns() - t0 > budget) {
       *abort = 1;
       report_error(st, kDevTimeout, site, blockIdx.x);
       return false;
+    }
+  }
+}
+
+// Whole warp: bounded wait until *cnt >= need, with acquire ordering for every
+// lane's later loads. Gives up on the CTA's abort flag or after the budget
+// (then records a timeout with the expert index and sets the abort flag).
+__device__ __forceinline__ bool wait_count(const uint32_t *cnt, uint32_t need, volatile int *abort, DevStatus *st,
+                                           uint32_t site, uint32_t detail, unsigned long long budget) {
+  unsigned long long t0 = 0;
+  for (unsigned it = 0;; ++it) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(cnt) : "memory");
+    if (__all_sync(0xffffffffu, v >= need)) return true;
+    if (__any_sync(0xffffffffu, *abort != 0)) return false;
+    if (it == 0) t0 = global_ns();
+    __nanosleep(64);
+    int late = 0;
+    if ((it & 15u) == 15u) late = global_ns() - t0 > budget ? 1 : 0;
+    if (__shfl_sync(0xffffffffu, late, 0)) {
+      if ((threadIdx.x & 31) == 0) {
+        *abort = 1;
+        report_error(st, kDevTimeout, site, detail);
+      }
+      return false;
+    }
+  }
+}
+
+// One thread: wait (bounded) for the last phase issued into each stage of a
+// ring, so that no copy into this CTA's shared memory is still in flight.
+__device__ __forceinline__ void drain_ring(uint64_t *full, const int *issued, int n) {
+  for (int s = 0; s < n; ++s) {
+    if (issued[s] <= 0) continue;
+    const uint32_t par = static_cast<uint32_t>(issued[s] - 1) & 1u;
+    const unsigned long long t0 = global_ns();
+    while (!mbar_try_wait(&full[s], par) && global_ns() - t0 < kWaitBudgetNs) {
     }
   }
 }
@@ -136,41 +192,6 @@ __device__ __forceinline__ void mma16816(float (&d)[4], uint32_t a0, uint32_t a1
       "{%0, %1, %2, %3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
-}
-
-// Grid barrier on {count, generation} with release/acquire atomics; returns
-// false if the wait ran out. The last CTA to arrive resets the count and bumps
-// the generation.
-__device__ bool grid_barrier(uint32_t *bar, DevStatus *st, int *ok_flag) {
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    uint32_t gen;
-    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(gen) : "l"(bar + 1) : "memory");
-    uint32_t arrived;
-    asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;" : "=r"(arrived) : "l"(bar) : "memory");
-    int ok = 1;
-    if (arrived == gridDim.x - 1) {
-      asm volatile("st.relaxed.gpu.global.u32 [%0], 0;" ::"l"(bar) : "memory");
-      asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(bar + 1) : "memory");
-    } else {
-      const unsigned long long t0 = global_ns();
-      unsigned it = 0;
-      while (true) {
-        uint32_t g;
-        asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(g) : "l"(bar + 1) : "memory");
-        if (g != gen) break;
-        __nanosleep(32);
-        if ((++it & 63u) == 0 && global_ns() - t0 > kWaitBudgetNs) {
-          report_error(st, kDevTimeout, 30, blockIdx.x);
-          ok = 0;
-          break;
-        }
-      }
-    }
-    *ok_flag = ok;
-  }
-  __syncthreads();
-  return *ok_flag != 0;
 }
 
 // Weight pointers of one expert id (E = the shared expert).
@@ -234,7 +255,7 @@ size_t small_t_smem_bytes(int T, int H, int k, int I, int Is) {
 
 bool small_t_fits(int T, int H, int k, int I, int Is, int num_sms) {
   return T >= 1 && T <= kSmallT && H % 256 == 0 && H / kRowBlock <= small_t_grid(num_sms) &&
-         small_t_smem_bytes(T, H, k, I, Is) <= 220 * 1024;
+         small_t_smem_bytes(T, H, k, I, Is) <= kStBudget;
 }
 
 __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs a) {
@@ -246,28 +267,39 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs
   const int g = lane >> 2, c = lane & 3;  // mma fragment coordinates
   __half *xs = reinterpret_cast<__half *>(dyn + L.x_off);  // [8][H + kXPad]
   float *red = reinterpret_cast<float *>(dyn + L.red_off); // [512 threads][8]
+  uint32_t *cand_key = reinterpret_cast<uint32_t *>(red);  // routing: [T][kCandPerToken]
+  int *cand_id = reinterpret_cast<int *>(red) + kSmallT * kCandPerToken;
   uint8_t *bring = dyn + L.b_off;
   uint8_t *dring = dyn + L.d_off;
   uint64_t *b_full = reinterpret_cast<uint64_t *>(dyn + L.bar_off);
   uint64_t *d_full = b_full + L.nb;
   volatile int *abort = &sh.abort;
-  __half *hb = reinterpret_cast<__half *>(a.hbuf);  // [T][k+1][Imax] fp16 scratch, operand order
+  __half *hb = a.hbuf;                               // [T][k+1][Imax] fp16 scratch, operand order
+  uint32_t *ready = a.sync;                          // [kMaxU] readiness counters
+  uint32_t *exit_count = a.sync + kMaxU;
+  uint32_t *router_count = a.sync + kMaxU + 1;       // CTAs whose router scores are published
+  const unsigned long long budget = a.wait_ns;
   const int Imax = L.Imax;
   const int nrb_sh = a.Is / kRowBlock;               // the shared expert's row blocks: the first units
+  const int nrb = a.I / kRowBlock;                   // row blocks of a routed expert
   const int n_dblk = H / kRowBlock;                  // phase-2 output blocks (one per CTA)
   const int hw = H / 8;                              // packed words per gate/up row
+  const bool has_dblk = blockIdx.x < n_dblk;
 
-  // ---- phase 0: set-up, routing, token staging, weight requests ------------------
+  // ---- set-up --------------------------------------------------------------------
   if (threadIdx.x == 0) {
     for (int s = 0; s < L.nb + L.nd; ++s) mbar_init(&b_full[s], 1);
     sh.abort = 0;
+    sh.ulist[0] = E;
     fence_barrier_init();
     fence_proxy_async_smem();
   }
   if (threadIdx.x < kSmallT) sh.xexp[threadIdx.x] = 0;
   if (threadIdx.x < kMaxExperts / 32) sh.bitmap[threadIdx.x] = 0;
+  if (threadIdx.x < 4) sh.b_iss[threadIdx.x] = 0;
   for (int i = threadIdx.x; i < kMaxU; i += kSTThreads) {
     sh.umask[i] = 0;
+    sh.d_iss[i] = 0;
 #pragma unroll
     for (int t = 0; t < kSmallT; ++t) sh.uslot[i][t] = -1;
   }
@@ -277,7 +309,9 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs
   // unit q of this CTA is global unit blockIdx.x + q * gridDim.x and uses ring
   // stage q % nb. A unit is six bulk copies (gate rows, up rows, their scales
   // and biases) from lanes 0..5 of the calling warp.
-  const int units_per_round = kSTWarps / L.ks;
+  // a round takes at most one unit per ring stage: every unit of a round has
+  // its copies issued before the round starts (the refill follows the round)
+  const int units_per_round = min(kSTWarps / L.ks, L.nb);
   auto issue_b = [&](int q) {  // all lanes of one warp
     const int unit = blockIdx.x + q * gridDim.x;
     int e, rb;
@@ -285,16 +319,21 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs
       e = E;
       rb = unit;
     } else {
-      e = sh.ulist[(unit - nrb_sh) / (a.I / kRowBlock)];
-      rb = (unit - nrb_sh) % (a.I / kRowBlock);
+      e = sh.ulist[1 + (unit - nrb_sh) / nrb];
+      rb = (unit - nrb_sh) % nrb;
     }
     const ExpertPtrs p = expert_ptrs(a, e);
-    uint8_t *st = bring + (q % L.nb) * L.b_stage;
+    const int s = q % L.nb;
+    uint8_t *st = bring + s * L.b_stage;
     const uint32_t pk = kRowBlock * (H / 2), sb = kRowBlock * (H / kGroup) * 2;
-    uint64_t *bar = &b_full[q % L.nb];
+    uint64_t *bar = &b_full[s];
     // the stage's only arrival is this expect-tx, so it cannot complete before
     // it, whatever order the copies land in
-    if (lane == 0) mbar_arrive_expect_tx(bar, 2 * pk + 4 * sb);
+    if (lane == 0) {
+      mbar_arrive_expect_tx(bar, 2 * pk + 4 * sb);
+      sh.b_iss[s] += 1;
+    }
+    __syncwarp();
     if (lane < 2) {
       const size_t row0 = static_cast<size_t>(lane) * p.Iu + rb * kRowBlock;
       bulk_g2s(st + lane * pk, p.packed + row0 * hw, pk, bar);
@@ -304,6 +343,7 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs
       const uint16_t *src = ((lane & 1) ? p.biases : p.scales) + row0 * (H / kGroup);
       bulk_g2s(st + 2 * pk + (lane - 2) * sb, src, sb, bar);
     }
+    __syncwarp();
   };
   // Phase-2 stage u % nd holds expert u's down rows [n0, n0 + 16): three copies,
   // ten experts per warp-wide step.
@@ -313,12 +353,14 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs
       const int sub = lane / 3, l = lane % 3, u = ub + sub;
       if (sub < 10 && u < u1) {
         const ExpertPtrs p = expert_ptrs(a, sh.ulist[u]);
-        uint8_t *st = dring + (u % L.nd) * L.d_stage;
+        const int s = u % L.nd;
+        uint8_t *st = dring + s * L.d_stage;
         const uint32_t pk = kRowBlock * (p.Iu / 2);
         const uint32_t sb = kRowBlock * (p.Iu / kGroup) * 2;
-        uint64_t *bar = &d_full[u % L.nd];
+        uint64_t *bar = &d_full[s];
         if (l == 0) {
           mbar_arrive_expect_tx(bar, pk + 2 * sb);
+          sh.d_iss[s] += 1;
           bulk_g2s(st, p.packed + static_cast<size_t>(2) * p.Iu * H / 8 + static_cast<size_t>(n0) * (p.Iu / 8), pk,
                    bar);
         } else {
@@ -330,65 +372,160 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs
     }
   };
 
-  const bool shared_first = blockIdx.x < nrb_sh;  // unit 0 is a shared-expert block: no routing needed
+  // ---- entry: the shared expert's copies need no routing -----------------------------
+  const bool shared_first = blockIdx.x < nrb_sh;  // unit 0 is a shared-expert block
   if (warp == 0 && shared_first) issue_b(0);
+  if (warp == 1 && has_dblk) issue_d_range(0, 1);  // expert u = 0 is the shared one
 
-  // tokens: the upper half of the CTA loads x (kept in registers) and reduces
-  // each token's max |x| while warps 0..T-1 route; a warp's 32 chunks of 8
-  // values belong to one token since H / 8 is a multiple of 32
+  // tokens: every thread loads its chunks of x now (kept in registers) so the
+  // loads overlap the logits loads of the routing below; a warp's 32 chunks of
+  // 8 values belong to one token since H / 8 is a multiple of 32
   constexpr int kXPer = kSmallT * 2048 / 8 / kSTThreads;  // cached chunks per thread (H <= 2048)
   const int nxc = T * hw;                                   // 8-value chunks of x
-  const int xt = (threadIdx.x + kSTThreads / 2) % kSTThreads;
   uint4 xv[kXPer];
 #pragma unroll
   for (int i = 0; i < kXPer; ++i) {
-    const int idx = xt + i * kSTThreads;
-    xv[i] = make_uint4(0, 0, 0, 0);
-    float m = 0.f;
-    if (idx < nxc) {
-      xv[i] = __ldg(reinterpret_cast<const uint4 *>(a.x) + idx);
-      m = bf16x8_absmax(xv[i]);
+    const int idx = threadIdx.x + i * kSTThreads;
+    xv[i] = idx < nxc ? __ldg(reinterpret_cast<const uint4 *>(a.x) + idx) : make_uint4(0, 0, 0, 0);
+  }
+
+  // ---- router scores, when they are computed here ---------------------------------------
+  // CTA b scores experts b, b + G, ... for every token: each (expert, token)
+  // dot product over H is split into 256-element slices over warps (fp32
+  // products of the bf16 operands), the slices summed in a fixed order. The
+  // scores go to global memory and are published with a release increment;
+  // every CTA then waits (bounded, acquire) until all scoring CTAs are done.
+  if (a.router_w) {
+    float *lw = const_cast<float *>(a.logits);
+    const int n_mine = blockIdx.x < static_cast<unsigned>(E) ? (E - 1 - blockIdx.x) / gridDim.x + 1 : 0;
+    const int nks = H / 256;
+    const int n_part = n_mine * T * nks;  // (expert, token, slice) partial sums of this CTA
+    for (int pw = warp; pw < n_part; pw += kSTWarps) {
+      const int pair = pw / nks, ks = pw % nks;
+      const int e = blockIdx.x + (pair / T) * gridDim.x, t = pair % T;
+      const uint4 xv8 = __ldg(reinterpret_cast<const uint4 *>(a.x + static_cast<size_t>(t) * H + ks * 256) + lane);
+      const uint4 wv8 = __ldg(reinterpret_cast<const uint4 *>(a.router_w + static_cast<size_t>(e) * H + ks * 256) + lane);
+      const uint32_t xs[4] = {xv8.x, xv8.y, xv8.z, xv8.w}, ws[4] = {wv8.x, wv8.y, wv8.z, wv8.w};
+      float acc = 0.f;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        acc = fmaf(__uint_as_float(xs[q] << 16), __uint_as_float(ws[q] << 16), acc);
+        acc = fmaf(__uint_as_float(xs[q] & 0xffff0000u), __uint_as_float(ws[q] & 0xffff0000u), acc);
+      }
+      acc = warp_sum(acc);
+      if (lane == 0) red[pw] = acc;
     }
-    m = warp_max(m);
-    const int idx0 = (xt & ~31) + i * kSTThreads;
+    __syncthreads();
+    for (int pair = threadIdx.x; pair < n_mine * T; pair += kSTThreads) {
+      float sum = 0.f;
+      for (int ks = 0; ks < nks; ++ks) sum += red[pair * nks + ks];
+      const int e = blockIdx.x + (pair / T) * gridDim.x, t = pair % T;
+      lw[static_cast<size_t>(t) * E + e] = sum;
+    }
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0 && n_mine > 0)
+      asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(router_count) : "memory");
+    const uint32_t n_scoring = static_cast<uint32_t>(min(E, static_cast<int>(gridDim.x)));
+    if (warp == 0) wait_count(router_count, n_scoring, abort, a.status, 43, 0, budget);
+    __syncthreads();
+  }
+
+  // ---- routing, step 1: the top k of each 32-expert slice of each token ----------------
+  // Order: larger float32 logit first, equal logits lower expert id first (a
+  // strict total order, since ids differ). One key per lane; a lane's rank in
+  // its slice is the number of lanes that precede it in that order, counted
+  // with shuffles. Lanes of rank < k write their candidate to position
+  // slice * k + rank of the token's candidate list (key 0: no expert there;
+  // it precedes nothing valid and is never among a token's top k, as k <= E).
+  const int nsl = (E + 31) / 32;
+  for (int un = warp; un < T * nsl; un += kSTWarps) {
+    const int t = un / nsl, sl = un % nsl, e = sl * 32 + lane;
+    // coherent load: with the router in this kernel, other CTAs wrote the scores
+    const uint32_t key = e < E ? float_key(__ldcg(a.logits + static_cast<size_t>(t) * E + e)) : 0u;
+    int rank = 0;
+#pragma unroll 8
+    for (int m = 0; m < 32; ++m) {
+      const uint32_t km = __shfl_sync(0xffffffffu, key, m);
+      rank += (km > key || (km == key && m < lane)) ? 1 : 0;
+    }
+    if (rank < k) {
+      cand_key[t * kCandPerToken + sl * k + rank] = key;
+      cand_id[t * kCandPerToken + sl * k + rank] = e;
+    }
+  }
+  // max |x| of each token (the power-of-two scale of its fp16 copy)
+#pragma unroll
+  for (int i = 0; i < kXPer; ++i) {
+    const int idx0 = (threadIdx.x & ~31) + i * kSTThreads;
+    const float m = warp_max(bf16x8_absmax(xv[i]));
     if (lane == 0 && idx0 < nxc && m > 0.f) atomicMax(&sh.xexp[idx0 / hw], __float_as_int(m));
   }
   for (int i0 = kXPer * kSTThreads; i0 < nxc; i0 += kSTThreads) {  // H > 2048
-    const int idx = xt + i0, idx0 = (xt & ~31) + i0;
+    const int idx = threadIdx.x + i0, idx0 = (threadIdx.x & ~31) + i0;
     float m = 0.f;
     if (idx < nxc) m = bf16x8_absmax(__ldg(reinterpret_cast<const uint4 *>(a.x) + idx));
     m = warp_max(m);
     if (lane == 0 && idx0 < nxc && m > 0.f) atomicMax(&sh.xexp[idx0 / hw], __float_as_int(m));
   }
+  __syncthreads();
+
+  // ---- routing, step 2: the token's top k among its slices' candidates --------------------
+  // The token's top k lie among the slices' top k. One lane per candidate:
+  // its rank among all nsl * k candidates of the token (broadcast reads of the
+  // list); the candidate of rank j < k is the token's j-th expert.
+  {
+    const int nc = nsl * k;
+    const int ngrp = (nc + 31) / 32;
+    for (int un = warp; un < T * ngrp; un += kSTWarps) {
+      const int t = un / ngrp, i = (un % ngrp) * 32 + lane;
+      const uint32_t *kl = cand_key + t * kCandPerToken;
+      const int *il = cand_id + t * kCandPerToken;
+      const uint32_t ck = i < nc ? kl[i] : 0u;
+      const int ci = i < nc ? il[i] : 0x7fffffff;
+      int rank = 0;
+      for (int m = 0; m < nc; ++m) {
+        const uint32_t km = kl[m];
+        rank += (km > ck || (km == ck && il[m] < ci)) ? 1 : 0;
+      }
+      if (i < nc && ck != 0u && rank < k) {
+        sh.ids[t][rank] = ci;
+        sh.wkey[t][rank] = ck;
+      }
+    }
+  }
+  __syncthreads();
+  // renormalised softmax weight of each chosen expert: the softmax over all E
+  // restricted to the chosen k and renormalised is exp(l_j - l_max) over the
+  // sum of those k terms (l_max = the first chosen logit)
   if (warp < T) {
-    int id;
-    float w;
-    warp_topk(a.logits + static_cast<size_t>(warp) * E, E, k, lane, id, w);
+    const int t = warp;
+    const float ex = lane < k ? expf(key_float(sh.wkey[t][lane]) - key_float(sh.wkey[t][0])) : 0.f;
+    const float z = warp_sum(ex);
     if (lane < k) {
-      sh.ids[warp][lane] = id;
-      sh.wt[warp][lane] = w;
+      const int id = sh.ids[t][lane];
+      sh.wt[t][lane] = ex / z;
       atomicOr(&sh.bitmap[id >> 5], 1u << (id & 31));
     }
   }
   __syncthreads();
-  // distinct experts: the rank of each set bit of the bitmap
+  // distinct experts: u = 1 + the rank of each set bit of the bitmap; u = 0 is shared
   if (warp == 0) {
     int before = 0;
 #pragma unroll
     for (int i = 0; i < kMaxExperts / 32; ++i) {
       const uint32_t wbits = sh.bitmap[i];
-      if ((wbits >> lane) & 1u) sh.ulist[before + __popc(wbits & ((1u << lane) - 1u))] = 32 * i + lane;
+      if ((wbits >> lane) & 1u) sh.ulist[1 + before + __popc(wbits & ((1u << lane) - 1u))] = 32 * i + lane;
       before += __popc(wbits);
     }
     if (lane == 0) {
-      sh.ulist[before] = E;
-      sh.umask[before] = (1u << T) - 1u;
-      for (int t = 0; t < T; ++t) sh.uslot[before][t] = static_cast<int8_t>(k);
+      sh.umask[0] = (1u << T) - 1u;
+      for (int t = 0; t < T; ++t) sh.uslot[0][t] = static_cast<int8_t>(k);
       sh.nU = before + 1;
     }
   } else if (threadIdx.x - 32 < T * k) {  // token/slot pairs: mask and slot of their expert
     const int f = threadIdx.x - 32, t = f / k, j = f % k, e = sh.ids[t][j];
-    int u = __popc(sh.bitmap[e >> 5] & ((1u << (e & 31)) - 1u));
+    int u = 1 + __popc(sh.bitmap[e >> 5] & ((1u << (e & 31)) - 1u));
     for (int i = 0; i < (e >> 5); ++i) u += __popc(sh.bitmap[i]);
     atomicOr(&sh.umask[u], 1u << t);
     sh.uslot[u][t] = static_cast<int8_t>(j);
@@ -401,14 +538,13 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs
   }
   __syncthreads();
   const int nU = sh.nU;
-  const int n_units = nrb_sh + (nU - 1) * (a.I / kRowBlock);
+  const int n_units = nrb_sh + (nU - 1) * nrb;
   const int my_units = blockIdx.x < n_units ? (n_units - 1 - blockIdx.x) / gridDim.x + 1 : 0;
-  const bool has_dblk = blockIdx.x < n_dblk;
   // the requests block their warp while many copies are outstanding, so each
-  // phase-1 unit (needed first) goes out from its own warp (2, 3, ...) and the
+  // phase-1 unit goes out from its own warp (2, 3, ...) and the routed experts'
   // down rows from warp 1, all in parallel
   if (warp == 1) {
-    if (has_dblk) issue_d_range(0, min(nU, L.nd));
+    if (has_dblk) issue_d_range(1, min(nU, L.nd));
   } else if (warp >= 2) {
     const int q = (shared_first ? 1 : 0) + warp - 2;
     if (q < min(my_units, L.nb)) issue_b(q);
@@ -416,12 +552,12 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs
   // stage the tokens: fp16 scaled by 2^-e in operand order; rows t >= T are zero
 #pragma unroll
   for (int i = 0; i < kXPer; ++i) {
-    const int idx = xt + i * kSTThreads;
+    const int idx = threadIdx.x + i * kSTThreads;
     if (idx < nxc)
       *reinterpret_cast<uint4 *>(xs + static_cast<size_t>(idx / hw) * (H + kXPad) + (idx % hw) * 8) =
           x_scaled_fp16(xv[i], sh.xexp[idx / hw]);
   }
-  for (int idx = xt + kXPer * kSTThreads; idx < nxc; idx += kSTThreads)
+  for (int idx = threadIdx.x + kXPer * kSTThreads; idx < nxc; idx += kSTThreads)
     *reinterpret_cast<uint4 *>(xs + static_cast<size_t>(idx / hw) * (H + kXPad) + (idx % hw) * 8) =
         x_scaled_fp16(__ldg(reinterpret_cast<const uint4 *>(a.x) + idx), sh.xexp[idx / hw]);
   for (int idx = nxc + threadIdx.x; idx < kSmallT * hw; idx += kSTThreads)
@@ -429,28 +565,28 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs
         make_uint4(0, 0, 0, 0);
   __syncthreads();
 
-  // ---- phase 1: gate/up ------------------------------------------------------------
+  // ---- gate/up ---------------------------------------------------------------------
   const int slot = warp / L.ks, kq = warp % L.ks;  // unit slot in a round, K slice of this warp
   const int rounds = (my_units + units_per_round - 1) / units_per_round;
+  const bool slot_used = slot < units_per_round;  // warps of an unused slot only join the barriers
   const int ng = H / kGroup;
   for (int r = 0; r < rounds; ++r) {
-    const int q = r * units_per_round + slot;
+    const int q = slot_used ? r * units_per_round + slot : my_units;
     float accg[4] = {0.f, 0.f, 0.f, 0.f}, accu[4] = {0.f, 0.f, 0.f, 0.f};
-    int u = 0, rb = 0;
+    int u = 0, rb = 0, unit = 0;
     if (q < my_units) {
-      const int unit = blockIdx.x + q * gridDim.x;
+      unit = blockIdx.x + q * gridDim.x;
       if (unit < nrb_sh) {
-        u = nU - 1;
+        u = 0;
         rb = unit;
       } else {
-        u = (unit - nrb_sh) / (a.I / kRowBlock);
-        rb = (unit - nrb_sh) % (a.I / kRowBlock);
+        u = 1 + (unit - nrb_sh) / nrb;
+        rb = (unit - nrb_sh) % nrb;
       }
       const int s = q % L.nb;
       int ok = 1;
-      if (lane == 0) ok = st_wait(&b_full[s], (q / L.nb) & 1u, abort, a.status, 40) ? 1 : 0;
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (ok) {
+      if (lane == 0) ok = st_wait(&b_full[s], (q / L.nb) & 1u, abort, a.status, 40, budget) ? 1 : 0;
+      if (__shfl_sync(0xffffffffu, ok, 0)) {
         const uint8_t *st = bring + s * L.b_stage;
         const uint32_t *pg = reinterpret_cast<const uint32_t *>(st);
         const uint32_t *pu = pg + kRowBlock * hw;
@@ -494,7 +630,8 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs
       rp[4 + i] = accu[i];
     }
     __syncthreads();
-    if (q < my_units && kq == 0) {
+    const bool live = __all_sync(0xffffffffu, *abort == 0);  // warp-uniform: the block below syncs the warp
+    if (q < my_units && kq == 0 && live) {
       float G[4] = {0.f, 0.f, 0.f, 0.f}, U[4] = {0.f, 0.f, 0.f, 0.f};
       for (int zz = 0; zz < L.ks; ++zz) {
         const float *zp = red + static_cast<size_t>((warp + zz) * 32 + lane) * 8;
@@ -515,100 +652,132 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs
           hb[(static_cast<size_t>(t) * (k + 1) + j) * Imax + (row & ~7) + kperm_dst(row & 7)] = __float2half_rn(hv);
         }
       }
+      // publish: the block's h values are visible before the count that says so
+      __threadfence();
+      __syncwarp();
+      if (lane == 0 && !(a.test_fault && unit == 0))
+        asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(ready + u) : "memory");
     }
     __syncthreads();
     // the stages this round used are free: refill them with the units nb ahead
-    if (warp == 0)
+    if (warp == 0 && __all_sync(0xffffffffu, *abort == 0))
       for (int zz = 0; zz < units_per_round; ++zz) {
         const int qn = r * units_per_round + zz + L.nb;
         if (qn < my_units) issue_b(qn);
       }
   }
 
-  // ---- grid barrier ------------------------------------------------------------------
-  if (!grid_barrier(a.barrier, a.status, &sh.ok)) return;
-
-  // ---- phase 2: down + combine -------------------------------------------------------
-  if (!has_dblk) return;
-  // copy the tokens' h (all slots) into the phase-1 ring, which is free now
-  __half *hs = reinterpret_cast<__half *>(bring);
-  const int hchunks = T * (k + 1) * Imax / 8;
-  for (int i = threadIdx.x; i < hchunks; i += kSTThreads)
-    reinterpret_cast<uint4 *>(hs)[i] = __ldcg(reinterpret_cast<const uint4 *>(hb) + i);
-  __syncthreads();
-  const int n0 = blockIdx.x * kRowBlock;
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};  // rows g, g+8; tokens 2c, 2c+1 (this warp's experts, ascending)
-  bool ok2 = true;
-  for (int base = 0; base < nU; base += L.nd) {
-    const uint32_t par = (base / L.nd) & 1u;
-    if (base > 0) {  // next pass: the ring's stages are free once every warp is done
-      __syncthreads();
-      if (warp == 0) issue_d_range(base, min(nU, base + L.nd));
-    }
-    for (int u = base + warp; u < min(nU, base + L.nd); u += kSTWarps) {
-      const int s = u % L.nd;
-      int ok = ok2 ? 1 : 0;
-      if (lane == 0 && ok) ok = st_wait(&d_full[s], par, abort, a.status, 41) ? 1 : 0;
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      ok2 = ok != 0;
-      if (!ok2) continue;
-      const int Iu = sh.ulist[u] == E ? a.Is : a.I;
-      const int iw = Iu / 8;  // packed words per down row
-      const uint8_t *st = dring + s * L.d_stage;
-      const uint32_t *pd = reinterpret_cast<const uint32_t *>(st);
-      const int ngd = Iu / kGroup;
-      const uint16_t *sd = reinterpret_cast<const uint16_t *>(st + kRowBlock * (Imax / 2));
-      const uint16_t *bd = sd + kRowBlock * ngd;
-      // B fragments: token g's h for this expert (zeros if g is not routed to it)
-      const int jg = (g < T) ? sh.uslot[u][g] : -1;
-      const __half *hrow = hs + (static_cast<size_t>(g) * (k + 1) + (jg < 0 ? 0 : jg)) * Imax;
-      float y[4] = {0.f, 0.f, 0.f, 0.f};
-      for (int wb = 0; wb < iw; wb += 16) {
-        const int w0 = wb + 4 * c;
-        const int grp = w0 / 8;
-        const __half2 s0 = bf16_to_half2_bcast(sd[g * ngd + grp]), b0 = bf16_to_half2_bcast(bd[g * ngd + grp]);
-        const __half2 s1 = bf16_to_half2_bcast(sd[(g + 8) * ngd + grp]),
-                      b1 = bf16_to_half2_bcast(bd[(g + 8) * ngd + grp]);
-        const uint4 wd0 = *reinterpret_cast<const uint4 *>(pd + g * iw + w0);
-        const uint4 wd1 = *reinterpret_cast<const uint4 *>(pd + (g + 8) * iw + w0);
-        const uint32_t ad0[4] = {wd0.x, wd0.y, wd0.z, wd0.w}, ad1[4] = {wd1.x, wd1.y, wd1.z, wd1.w};
+  // ---- down + combine ----------------------------------------------------------------
+  if (has_dblk) {
+    const int n0 = blockIdx.x * kRowBlock;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};  // rows g, g+8; tokens 2c, 2c+1 (this warp's experts, ascending)
+    bool ok2 = __all_sync(0xffffffffu, *abort == 0);
+    for (int base = 0; base < nU; base += L.nd) {
+      const uint32_t par = (base / L.nd) & 1u;
+      if (base > 0) {  // next pass: the ring's stages are free once every warp is done
+        __syncthreads();
+        if (warp == 0 && __all_sync(0xffffffffu, *abort == 0)) issue_d_range(base, min(nU, base + L.nd));
+      }
+      for (int u = base + warp; u < min(nU, base + L.nd); u += kSTWarps) {
+        if (!ok2) break;
+        const int s = u % L.nd;
+        int okw = 1;
+        if (lane == 0) okw = st_wait(&d_full[s], par, abort, a.status, 41, budget) ? 1 : 0;
+        ok2 = __shfl_sync(0xffffffffu, okw, 0) != 0;
+        if (!ok2) break;
+        const int Iu = u == 0 ? a.Is : a.I;
+        // every row block of expert u has published its h
+        ok2 = wait_count(ready + u, static_cast<uint32_t>(Iu / kRowBlock), abort, a.status, 42, u, budget);
+        if (!ok2) break;
+        const int iw = Iu / 8;  // packed words per down row
+        const uint8_t *st = dring + s * L.d_stage;
+        const uint32_t *pd = reinterpret_cast<const uint32_t *>(st);
+        const int ngd = Iu / kGroup;
+        const uint16_t *sd = reinterpret_cast<const uint16_t *>(st + kRowBlock * (Imax / 2));
+        const uint16_t *bd = sd + kRowBlock * ngd;
+        // B fragments: token g's h for this expert (zeros if g is not routed to
+        // it), read from L2 (written by other CTAs of this launch)
+        const int jg = (g < T) ? sh.uslot[u][g] : -1;
+        const __half *hrow = hb + (static_cast<size_t>(g) * (k + 1) + (jg < 0 ? 0 : jg)) * Imax;
+        float y[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int wb = 0; wb < iw; wb += 32) {  // two 16-word blocks per pass: 8 h loads in flight
+          uint4 hv[2][4];
 #pragma unroll
-        for (int p = 0; p < 4; ++p) {
-          uint4 hbv = make_uint4(0, 0, 0, 0);
-          if (jg >= 0) hbv = *reinterpret_cast<const uint4 *>(hrow + (w0 + p) * 8);
-          const uint4 d0 = dequant_word(ad0[p], s0, b0), d1 = dequant_word(ad1[p], s1, b1);
-          mma16816(y, d0.x, d1.x, d0.y, d1.y, hbv.x, hbv.y);
-          mma16816(y, d0.z, d1.z, d0.w, d1.w, hbv.z, hbv.w);
+          for (int b2 = 0; b2 < 2; ++b2)
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+              const int w = wb + 16 * b2 + 4 * c + p;
+              hv[b2][p] = (jg >= 0 && w < iw) ? __ldcg(reinterpret_cast<const uint4 *>(hrow + w * 8))
+                                               : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+          for (int b2 = 0; b2 < 2; ++b2) {
+            const int w0 = wb + 16 * b2 + 4 * c;
+            if (wb + 16 * b2 >= iw) break;
+            const int grp = w0 / 8;
+            const __half2 s0 = bf16_to_half2_bcast(sd[g * ngd + grp]), b0 = bf16_to_half2_bcast(bd[g * ngd + grp]);
+            const __half2 s1 = bf16_to_half2_bcast(sd[(g + 8) * ngd + grp]),
+                          b1 = bf16_to_half2_bcast(bd[(g + 8) * ngd + grp]);
+            const uint4 wd0 = *reinterpret_cast<const uint4 *>(pd + g * iw + w0);
+            const uint4 wd1 = *reinterpret_cast<const uint4 *>(pd + (g + 8) * iw + w0);
+            const uint32_t ad0[4] = {wd0.x, wd0.y, wd0.z, wd0.w}, ad1[4] = {wd1.x, wd1.y, wd1.z, wd1.w};
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
+              const uint4 d0 = dequant_word(ad0[p], s0, b0), d1 = dequant_word(ad1[p], s1, b1);
+              mma16816(y, d0.x, d1.x, d0.y, d1.y, hv[b2][p].x, hv[b2][p].y);
+              mma16816(y, d0.z, d1.z, d0.w, d1.w, hv[b2][p].z, hv[b2][p].w);
+            }
+          }
+        }
+        // weight each token's column by its routing weight (1 for the shared expert) and 2^(2e)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int t = 2 * c + (i & 1);
+          if (t < T && ((sh.umask[u] >> t) & 1u)) {
+            const int j = sh.uslot[u][t];
+            const float wgt = (j == k) ? 1.0f : sh.wt[t][j];
+            acc[i] += wgt * ldexpf(y[i], 2 * sh.xexp[t]);
+          }
         }
       }
-      // weight each token's column by its routing weight (1 for the shared expert) and 2^(2e)
+    }
+    float *rp = red + static_cast<size_t>(threadIdx.x) * 8;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) rp[i] = acc[i];
+    __syncthreads();
+    // warps' contributions summed in warp order, one rounding; 16 rows x T tokens
+    if (warp == 0) {
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int t = 2 * c + (i & 1);
-        if (t < T && ((sh.umask[u] >> t) & 1u)) {
-          const int j = sh.uslot[u][t];
-          const float wgt = (j == k) ? 1.0f : sh.wt[t][j];
-          acc[i] += wgt * ldexpf(y[i], 2 * sh.xexp[t]);
+        const int n = n0 + g + (i >> 1) * 8;
+        if (t < T) {
+          float o = 0.f;
+          for (int zz = 0; zz < kSTWarps; ++zz) o += red[static_cast<size_t>(zz * 32 + lane) * 8 + i];
+          if (a.residual) o += bf16_bits_to_float(a.residual[static_cast<size_t>(t) * H + n]);
+          a.out[static_cast<size_t>(t) * H + n] = float_to_bf16_bits(o);
         }
       }
     }
   }
-  float *rp = red + static_cast<size_t>(threadIdx.x) * 8;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) rp[i] = acc[i];
+
+  // ---- exit ----------------------------------------------------------------------------
   __syncthreads();
-  // warps' contributions summed in warp order, one rounding; 16 rows x T tokens
-  if (warp == 0) {
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int t = 2 * c + (i & 1);
-      const int n = n0 + g + (i >> 1) * 8;
-      if (t < T) {
-        float o = 0.f;
-        for (int zz = 0; zz < kSTWarps; ++zz) o += red[static_cast<size_t>(zz * 32 + lane) * 8 + i];
-        if (a.residual) o += bf16_bits_to_float(a.residual[static_cast<size_t>(t) * H + n]);
-        a.out[static_cast<size_t>(t) * H + n] = float_to_bf16_bits(o);
-      }
+  if (threadIdx.x == 0) {
+    // after a wait gave up, copies may still be in flight: they land before the
+    // CTA leaves (without one, every issued stage has been waited on)
+    if (*abort) {
+      drain_ring(b_full, sh.b_iss, L.nb);
+      drain_ring(d_full, sh.d_iss, L.nd);
+    }
+    // every CTA has finished reading the counters once all have arrived here:
+    // the last one clears them for the next launch on the stream
+    uint32_t arrived;
+    asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;" : "=r"(arrived) : "l"(exit_count) : "memory");
+    if (arrived == gridDim.x - 1) {
+      for (int u = 0; u < kMaxU; ++u) ready[u] = 0u;
+      *router_count = 0u;
+      *exit_count = 0u;
     }
   }
 }
@@ -616,8 +785,9 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs
 cudaError_t launch_small_t(const SmallTArgs &a, int num_sms, cudaStream_t s) {
   const StLayout L = st_layout(a.H, a.I, a.Is, a.T, a.k);
   const size_t smem = L.bytes;
-  cudaError_t err = cudaFuncSetAttribute(small_t_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+  // the limit is raised to the most any layout takes, once per device
+  static std::atomic<uint64_t> smem_set{0};
+  cudaError_t err = gemm::ensure_smem_limit(small_t_kernel, static_cast<int>(kStBudget), smem_set);
   if (err != cudaSuccess) return err;
   SmallTArgs args = a;
   void *params[] = {&args};

@@ -75,7 +75,27 @@ enum {
   /* Route every batch through the grouped-GEMM path, even T <= 8 (testing). */
   MOE_FLAG_FORCE_GROUPED = 1,
   /* Route every batch through the small-T path (T <= 8 only; testing). */
-  MOE_FLAG_FORCE_SMALL_T = 2
+  MOE_FLAG_FORCE_SMALL_T = 2,
+  /* Range-check, on the device, every index the kernels read from the
+   * routing artefacts: each grouped-GEMM work item (expert, weight-row block,
+   * first activation row and row count, hence every TMA coordinate derived
+   * from it) and each inverse-permutation entry the combine reads. A bad one
+   * is skipped and recorded as MOE_ERR_DEVICE_BOUNDS for moe_status_sync;
+   * nothing traps. The checks cost a few instructions per work item. */
+  MOE_FLAG_DEBUG = 4,
+  /* Testing only: the plan's first small-T launch makes one of its bounded
+   * waits run out (row block 0 of the shared expert does not announce that
+   * its SwiGLU output is ready) with a 2 ms budget instead of 2 s; every
+   * other wait of that launch is bounded too and the launch ends normally.
+   * moe_status_sync then reports MOE_ERR_DEVICE_TIMEOUT and clears the
+   * state, and later calls on the plan run normally. */
+  MOE_FLAG_TEST_WAIT_TIMEOUT = 8,
+  /* Launch the grouped path's kernels in plain stream order. By default each
+   * of them goes out with programmatic dependent launch: it may be scheduled
+   * while the kernel before it on the stream finishes, runs its prologue
+   * (barrier set-up, tensor-memory allocation) and waits for that kernel to
+   * complete before it touches global memory. Results are identical. */
+  MOE_FLAG_NO_PDL = 16
 };
 
 /* Device pointers of one layer's weights, for moe_stack_forward. */
@@ -90,12 +110,18 @@ typedef struct {
 
 /*
  * Create a plan for batches of up to T_max tokens.
- *   hidden (H), inter (I), shared_inter (Is): multiples of 128.
+ * The pages say only that the engine keeps execution plans and chooses its
+ * kernels per shape ("Perplexity open sources Lily...", section
+ * "Requirements and model layout"); a plan here is the sizes plus the
+ * device workspace of the routing, the grouped GEMMs and the small-T kernel.
+ *   hidden (H), inter (I), shared_inter (Is): multiples of 128 (a multiple of
+ *   the pages' 64-weight group, as the tensor-core tiles take whole 128-row
+ *   blocks of every weight matrix; the small-T kernel also needs H % 256 == 0).
  *   n_experts (E): 1..256; top_k (k): 1..min(E, 16).
  * Allocates the device workspace on the current device (cudaMalloc); the
  * plan owns it until moe_plan_destroy. *out receives the plan.
- * Errors: MOE_ERR_INVALID_ARG (sizes), MOE_ERR_NO_DEVICE, MOE_ERR_CUDA
- * (allocation failed; nothing is leaked).
+ * Errors: MOE_ERR_INVALID_ARG (sizes, unknown or conflicting flags),
+ * MOE_ERR_NO_DEVICE, MOE_ERR_CUDA (allocation failed; nothing is leaked).
  */
 moe_status moe_plan(int T_max, int hidden, int n_experts, int top_k, int inter,
                     int shared_inter, int flags, moe_plan_t **out);
@@ -107,7 +133,12 @@ moe_status moe_plan_destroy(moe_plan_t *plan);
 int64_t moe_plan_workspace_bytes(const moe_plan_t *plan);
 
 /*
- * One MoE layer for T tokens (0 <= T <= T_max).
+ * One MoE layer for T tokens (0 <= T <= T_max): the top-k routing over all
+ * experts plus the always-on shared expert ("Perplexity open sources
+ * Lily...", section "Requirements and model layout"), with the 4-bit weights
+ * dequantised one tile at a time inside the grouped expert GEMMs and fp32
+ * accumulation (aioga.com record, article body paragraph 4) and the routing
+ * kept on the GPU in one stream (same record, paragraph 5).
  *   x_bf16        [T, H] bfloat16 input activations.
  *   router_logits [T, E] float32 router scores (finite values).
  *   packed_w, scales, biases, shared_*: the layer's weights (layout above).
@@ -126,6 +157,35 @@ moe_status moe_forward(moe_plan_t *plan, int T, const void *x_bf16,
                        moe_stream_t stream);
 
 /*
+ * One MoE layer whose router scores are computed here instead of being
+ * passed in: the router "scores 256 experts and picks eight" ("Perplexity
+ * open sources Lily...", section "Requirements and model layout"), so
+ *   logits[t, e] = sum_h x[t, h] * router_w[e, h]
+ * in float32 (bfloat16 operands, float32 accumulation), then the layer of
+ * moe_forward on those logits.
+ *   router_w_bf16 [E, H] bfloat16 router weight (device, 16-byte aligned).
+ * Other arguments as moe_forward. T <= 8 computes the scores inside the
+ * fused small-T kernel (each CTA a slice of the experts, published to the
+ * others through the plan's workspace); larger T runs a tensor-core router
+ * kernel ahead of the routing. The selection compares the float32 scores, so
+ * two experts whose exact scores lie within float32 rounding of each other
+ * may be ordered either way.
+ */
+moe_status moe_forward_router(moe_plan_t *plan, int T, const void *x_bf16,
+                              const void *router_w_bf16, const uint32_t *packed_w,
+                              const void *scales, const void *biases,
+                              const uint32_t *shared_packed_w, const void *shared_scales,
+                              const void *shared_biases, void *out_bf16,
+                              moe_stream_t stream);
+
+/*
+ * The router scores alone (the tensor-core router kernel), for checks:
+ *   logits_out [T, E] float32 (device) = x [T, H] . router_w [E, H]^T.
+ */
+moe_status moe_router_logits(moe_plan_t *plan, int T, const void *x_bf16, const void *router_w_bf16,
+                             float *logits_out, moe_stream_t stream);
+
+/*
  * moe_forward with HOST activations: x_bf16_host, router_logits_host and
  * out_bf16_host are host pointers (pinned memory gives asynchronous copies);
  * the weights are device pointers. Copies the inputs into the plan's device
@@ -140,7 +200,10 @@ moe_status moe_forward_host(moe_plan_t *plan, int T, const void *x_bf16_host,
                             moe_stream_t stream);
 
 /*
- * n_layers stacked MoE layers with a residual, in place:
+ * n_layers stacked MoE layers with a residual, in place (the pages' model has
+ * 40 such layers, "Perplexity open sources Lily...", section "Requirements
+ * and model layout"; the engine runs them back to back on the GPU without
+ * host round trips, aioga.com record, article body paragraphs 5-6):
  *   x <- bfloat16(x + moe_l(x)) for l = 0..n_layers-1,
  * the residual add fused into each layer's combine (one rounding per layer).
  *   x_inout_bf16 [T, H] device, logits [n_layers, T, E] device float32,
@@ -165,7 +228,10 @@ moe_status moe_route(moe_plan_t *plan, int T, const float *logits, int32_t *ids,
                      float *w, int32_t *offsets, int32_t *perm, moe_stream_t stream);
 
 /*
- * Wait for the stream, then read and clear the plan's device status word.
+ * Wait for the stream, then read the plan's device status word. After a
+ * device error it also clears the status word and the small-T kernel's
+ * counters, so the plan can be used again. The pages describe no error
+ * reporting; this is the library's own.
  * Returns MOE_OK, MOE_ERR_DEVICE_TIMEOUT, MOE_ERR_DEVICE_BOUNDS or
  * MOE_ERR_CUDA (with the CUDA error in moe_last_error()).
  */
@@ -189,7 +255,8 @@ enum {
   MOE_KERNEL_DOWN = 5,
   MOE_KERNEL_COMBINE = 6,
   MOE_KERNEL_SMALL_T = 7,
-  MOE_KERNEL_COUNT = 8
+  MOE_KERNEL_ROUTER = 8,
+  MOE_KERNEL_COUNT = 9
 };
 moe_status moe_profile_enable(moe_plan_t *plan, int max_launches);
 moe_status moe_profile_read(moe_plan_t *plan, moe_stream_t stream, double *ms, int32_t *launches);
@@ -199,22 +266,27 @@ moe_status moe_profile_read(moe_plan_t *plan, moe_stream_t stream, double *ms, i
  * The source pages describe no such call; it exists for callers that
  * cannot call cudaMalloc (code running inside an allocator or memory-pool
  * callback, runtimes that reserve all device memory up front), and so cannot
- * create a plan. Its scratch memory (SwiGLU outputs, grid-barrier words,
- * status word) lives in one static __device__ array of 512 KiB inside the
- * library, which every GPU that loads the library holds until the process
- * exits; the caller passes only inputs and outputs, as for moe_forward.
- *   Sizes: as moe_plan, plus 8 * (top_k + 1) * max(inter, shared_inter) * 4
- *   bytes must fit in 512 KiB - 256 bytes; larger layers get
- *   MOE_ERR_UNSUPPORTED, T > 8 gets MOE_ERR_INVALID_ARG.
- *   status_out: optional device pointer to 16 bytes that receive the device
- *   status word of this call ({code, site, detail, 0}; code 0 = OK).
+ * create a plan. Its scratch memory (SwiGLU outputs, the kernel's readiness
+ * counters, status word) lives in one static __device__ array of 512 KiB
+ * inside the library, which every GPU that loads the library holds until the
+ * process exits; the caller passes only inputs and outputs, as for
+ * moe_forward, and gets the same result bit for bit.
+ *   Sizes: hidden a multiple of 256 (at most 16384), inter and shared_inter
+ *   multiples of 128 (at most 8192), top_k <= min(n_experts, 16),
+ *   n_experts <= 256; and the fp16 SwiGLU outputs,
+ *   8 * (top_k + 1) * max(inter, shared_inter) * 2 bytes, must fit in
+ *   512 KiB - 1280 bytes. Larger layers get MOE_ERR_UNSUPPORTED, T > 8 and
+ *   bad sizes MOE_ERR_INVALID_ARG.
+ *   status_out: optional device pointer to 16 bytes (16-byte aligned) that
+ *   receive the device status word of this call ({code, site, detail, 0};
+ *   code 0 = OK); a call with T == 0 writes a zero status there.
  * The first call on a device looks up the array's device address (once per
- * device, with that device current); make that first call before capturing
- * the stream into a CUDA graph. Each call clears the barrier and status words
- * on the stream and calls no cudaMalloc, cudaFree or allocating library
- * routine. All calls on one device share that device's copy of the array,
- * so calls that overlap on the GPU (for example on two streams) race:
- * serialise them on one stream.
+ * device, with that device current; a failed lookup is retried by the next
+ * call); make that first call before capturing the stream into a CUDA graph.
+ * Each call clears the counters and the status word on the stream and calls
+ * no cudaMalloc, cudaFree or allocating library routine. All calls on one
+ * device share that device's copy of the array, so calls that overlap on the
+ * GPU (for example on two streams) race: serialise them on one stream.
  */
 moe_status moe_forward_small_t_noalloc(int T, int hidden, int n_experts, int top_k, int inter,
                                        int shared_inter, const void *x_bf16,

@@ -108,14 +108,22 @@ def test_forward_mid_size_ragged():
     check_output(_forward(_plan(inp), inp), oracle.moe_forward(inp), "mid")
 
 
-@pytest.mark.parametrize("name,nrows", [("prefill", 96), ("zipf", 96)])
-def test_forward_full_size_sampled_rows(name, nrows):
+@pytest.mark.parametrize("name", ["prefill", "zipf"])
+def test_forward_full_size_every_row(name):
+    """Every token row of the full-size layer against the oracle (the by-expert
+    form of the same definition). At Zipf T=4096 this covers the tail experts
+    whose few tokens fill ragged, mostly empty tiles."""
     inp = workload(name)
     got = _forward(_plan(inp), inp)
-    rng = np.random.default_rng(99)
-    rows = np.unique(np.concatenate([[0, inp.T - 1], rng.choice(inp.T, nrows - 2, replace=False)]))
-    ref = oracle.moe_forward(inp, x=inp.x[rows], logits=inp.logits[rows])
-    check_output(got[rows], ref, name)
+    check_output(got, oracle.moe_forward_by_expert(inp), name)
+
+
+def test_zipf_tail_experts_have_ragged_groups():
+    """The Zipf layer does route some experts only a handful of tokens (the
+    ragged tiles the previous test covers) and leaves others untouched."""
+    inp = workload("zipf")
+    counts = oracle.route(inp.logits, inp.k)[2]
+    assert (counts == 0).sum() > 100 and ((counts > 0) & (counts < 16)).sum() >= 3
 
 
 @pytest.mark.parametrize("T", [1, 2, 3, 5, 8, 9])
@@ -138,6 +146,15 @@ def test_small_batch_hidden_sizes(H, T):
     """Hidden sizes whose per-warp K slices of the small-batch kernel are 1, 2 and 5 blocks of 128."""
     inp = synth.make_layer(T, H, 16, 2, 128, 256, seed=300 + H + T, logit_std=1.0)
     check_output(_forward(_plan(inp), inp), oracle.moe_forward(inp), f"H={H} T={T}")
+
+
+@pytest.mark.parametrize("H", [256, 512])
+def test_small_batch_many_units_per_block(H):
+    """T=8 over 256 experts: up to 65 distinct experts, so each CTA of the
+    small-batch kernel takes many 16-row units and recycles both rings; at
+    these hidden sizes a round could hold more units than ring stages."""
+    inp = synth.make_layer(8, H, 256, 8, 512, 512, seed=400 + H, logit_std=2.0)
+    check_output(_forward(_plan(inp), inp), oracle.moe_forward(inp), f"many units H={H}")
 
 
 def test_one_expert_takes_every_token():
@@ -198,3 +215,61 @@ def test_invalid_arguments_enqueue_nothing():
     with pytest.raises(api.MoEError):
         api.moe_forward(plan.handle, inp.T, x, logits, *_layer(inp).args(), x)  # out aliases x
     plan.status_sync()
+
+
+# ----------------------------------------------------------------------------
+# MOE_FLAG_DEBUG range checks and the bounded waits
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("case", ["tiny", "mid", "zipf", "decode"])
+def test_debug_range_checks_pass_on_valid_runs(case):
+    """With every work item and inverse-permutation entry range-checked on the
+    device, a valid layer reports no error and still matches the oracle."""
+    if case == "mid":
+        inp = synth.make_layer(300, 512, 32, 4, 256, 384, seed=21, logit_std=1.0)
+    else:
+        inp = workload(case)
+    plan = _plan(inp, flags=api.MOE_FLAG_DEBUG | (api.MOE_FLAG_FORCE_GROUPED if case == "decode" else 0))
+    got = _forward(plan, inp)  # status_sync raises on any recorded error
+    ref = oracle.moe_forward_by_expert(inp) if inp.T > 64 else oracle.moe_forward(inp)
+    check_output(got, ref, f"debug {case}")
+
+
+def test_bounded_wait_runs_out_and_the_plan_recovers():
+    """The test flag makes one wait of the plan's first small-T launch run out
+    (row block 0 of the shared expert never announces its output) under a
+    2 ms budget: nothing faults, every other wait is bounded, the launch ends
+    and moe_status_sync reports the timeout. The next launch on the same plan
+    runs normally and matches the oracle."""
+    inp = synth.make_layer(1, 2048, 256, 8, 512, 512, seed=601, logit_std=2.0)
+    layer = _layer(inp)
+    plan = _plan(inp, flags=api.MOE_FLAG_TEST_WAIT_TIMEOUT)
+    x, logits = to_device(inp)
+    plan.forward(x, logits, layer)
+    with pytest.raises(api.MoEError) as ei:
+        plan.status_sync()
+    assert ei.value.status == -4 and "wait ran out" in str(ei.value)
+    for _ in range(2):
+        out = plan.forward(x, logits, layer)
+        plan.status_sync()
+        check_output(out.cpu().numpy(), oracle.moe_forward(inp), "after the timeout")
+
+
+def test_programmatic_dependent_launch_gives_identical_results():
+    """Three stacked layers of the grouped path, with the default programmatic
+    dependent launch and in plain stream order: bit-identical outputs."""
+    inp = synth.make_layer(300, 512, 32, 4, 256, 384, seed=23, logit_std=1.0)
+    layer = _layer(inp)
+    rng = np.random.default_rng(5)
+    logits = np.stack([synth.draw_logits(rng, inp.T, inp.E, inp.k, 1.0, None) for _ in range(3)])
+    dlog = torch.from_numpy(logits).cuda()
+    outs = []
+    for flags in (0, api.MOE_FLAG_NO_PDL):
+        plan = _plan(inp, flags=flags)
+        x = torch.from_numpy(inp.x.view(np.int16)).cuda()
+        torch.cuda.synchronize()
+        plan.stack_forward(x, dlog, [layer] * 3)
+        plan.status_sync()
+        outs.append(x.cpu().numpy())
+        plan.close()
+    assert np.array_equal(outs[0], outs[1])
