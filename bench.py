@@ -144,10 +144,26 @@ def touched_experts(inp):
     return len(np.unique(order)) + 1
 
 
-def roofline_numbers(inp, peaks):
+# Layers whose logits come from a router weight (the router scores computed by
+# the library ahead of the routing), on the sizes and seeds of a base workload.
+ROUTER_WORKLOADS = {"decode_router": "decode", "prefill_router": "prefill"}
+
+
+def make_inputs(name):
+    """(LayerInputs, router weight or None) of a benchmark workload."""
+    if name in ROUTER_WORKLOADS:
+        wl = synth.WORKLOADS[ROUTER_WORKLOADS[name]]
+        return synth.make_router_layer(wl.T, wl.H, wl.E, wl.k, wl.I, wl.Is, wl.seed, wl.logit_std)
+    return synth.make_workload(name), None
+
+
+def roofline_numbers(inp, peaks, router_w=None):
     ex = touched_experts(inp)
     wbytes = ex * synth.expert_bytes(inp.H, inp.I)
     flops = synth.layer_flops(inp.T, inp.H, inp.k, inp.I)
+    if router_w is not None:  # the router weight is read once, its scores are a dense product
+        wbytes += router_w.size * 2
+        flops += 2.0 * inp.T * inp.E * inp.H
     t_hbm = wbytes / (peaks["hbm_gbs"] * 1e9)
     t_tc = flops / (peaks["bf16_tflops"] * 1e12)
     return dict(touched=ex, weight_bytes=wbytes, flops=flops, t_hbm=t_hbm, t_tc=t_tc,
@@ -263,9 +279,19 @@ def run_gpu(args, rank, world, local_rank):
     def measure(name, steps, warmup):
         if name == "stack":
             return measure_stack(steps, warmup)
-        inp = synth.make_workload(name)
-        rf = roofline_numbers(inp, peaks)
+        inp, router_w = make_inputs(name)
         base = api.DeviceLayer.from_inputs(inp, dev)
+        x = torch.from_numpy(inp.x.view(np.int16)).to(dev)
+        plan = api.Plan(inp.T, inp.H, inp.E, inp.k, inp.I, inp.Is)
+        wr = None
+        if router_w is not None:
+            # the touched experts follow the library's own scores
+            wr = torch.from_numpy(router_w.view(np.int16)).to(dev)
+            lg = torch.empty((inp.T, inp.E), dtype=torch.float32, device=dev)
+            api.moe_router_logits(plan.handle, inp.T, x, wr, lg)
+            plan.status_sync()
+            inp.logits = lg.cpu().numpy()
+        rf = roofline_numbers(inp, peaks, router_w)
         layer_bytes = sum(t.numel() * t.element_size() for t in base.args())
         touched = max(rf["weight_bytes"], 1)
         n_rep = int(min(32, max(2, -(-4 * l2 // touched))))
@@ -274,15 +300,16 @@ def run_gpu(args, rank, world, local_rank):
             n_rep = args.replicas
         reps = [base] + [api.DeviceLayer(*[t.clone() for t in base.args()]) for _ in range(n_rep - 1)]
         rep_ptrs = [[t.data_ptr() for t in r.args()] for r in reps]
-        x = torch.from_numpy(inp.x.view(np.int16)).to(dev)
         logits = torch.from_numpy(inp.logits).to(dev)
         out = torch.empty_like(x)
-        plan = api.Plan(inp.T, inp.H, inp.E, inp.k, inp.I, inp.Is)
         stream = torch.cuda.Stream(dev)  # graphs cannot be captured on the default stream
         torch.cuda.set_stream(stream)
 
         def step(i):
-            api.moe_forward(plan.handle, inp.T, x, logits, *rep_ptrs[i % n_rep], out, stream)
+            if wr is None:
+                api.moe_forward(plan.handle, inp.T, x, logits, *rep_ptrs[i % n_rep], out, stream)
+            else:
+                api.moe_forward_router(plan.handle, inp.T, x, wr, *rep_ptrs[i % n_rep], out, stream)
 
         for i in range(warmup):
             step(i)
@@ -320,7 +347,26 @@ def run_gpu(args, rank, world, local_rank):
         plan.status_sync(stream)
         ms_step = ms_region / timed_steps
         tokens_s = whole_job_tokens_s(inp.T, world, ms_step)
-        # end to end through the host-buffer entry point (pinned host memory)
+        e2e_tok_s = None
+        if wr is None:
+            e2e_tok_s = measure_e2e(inp, plan, rep_ptrs, n_rep, stream, ms_step)
+        achieved_gbs = rf["weight_bytes"] / (ms_step * 1e-3) / 1e9
+        achieved_tf = rf["flops"] / (ms_step * 1e-3) / 1e12
+        res = dict(workload=name, T=inp.T, ms_per_step=ms_step, tokens_s=tokens_s, rf=rf,
+                   achieved_gbs=achieved_gbs, achieved_tflops=achieved_tf, n_rep=n_rep,
+                   graph=True, timed_steps=timed_steps, regions=[round(t, 4) for t in all_regions],
+                   clocks=clk.summary(), e2e_tokens_s=e2e_tok_s,
+                   h2d=inp.T * inp.H * 2 + inp.T * inp.E * 4, d2h=inp.T * inp.H * 2,
+                   launches=launches_per_step * timed_steps, inp=inp, prof=prof,
+                   launches_per_step=launches_per_step)
+        del g
+        plan.close()
+        del reps, base
+        torch.cuda.empty_cache()
+        return res
+
+    def measure_e2e(inp, plan, rep_ptrs, n_rep, stream, ms_step):
+        """End to end through the host-buffer entry point (pinned host memory)."""
         xh = torch.from_numpy(inp.x.view(np.int16)).pin_memory()
         lh = torch.from_numpy(inp.logits).pin_memory()
         oh = torch.empty_like(xh).pin_memory()
@@ -335,25 +381,12 @@ def run_gpu(args, rank, world, local_rank):
         e2e_s = (time.perf_counter() - t0) / n_e2e
         e2e_s = reduce_max(e2e_s, world, dev)
         plan.status_sync(stream)
-        achieved_gbs = rf["weight_bytes"] / (ms_step * 1e-3) / 1e9
-        achieved_tf = rf["flops"] / (ms_step * 1e-3) / 1e12
-        res = dict(workload=name, T=inp.T, ms_per_step=ms_step, tokens_s=tokens_s, rf=rf,
-                   achieved_gbs=achieved_gbs, achieved_tflops=achieved_tf, n_rep=n_rep,
-                   graph=True, timed_steps=timed_steps, regions=[round(t, 4) for t in all_regions],
-                   clocks=clk.summary(), e2e_tokens_s=inp.T * world / e2e_s,
-                   h2d=inp.T * inp.H * 2 + inp.T * inp.E * 4, d2h=inp.T * inp.H * 2,
-                   launches=launches_per_step * timed_steps, inp=inp, prof=prof,
-                   launches_per_step=launches_per_step)
-        del g
-        plan.close()
-        del reps, base
-        torch.cuda.empty_cache()
-        return res
+        return inp.T * world / e2e_s
 
     main = measure(args.workload, args.steps, args.warmup)
     extra = {}
     if not args.no_extra and world == 1:
-        for name in ("prefill", "zipf", "stack"):
+        for name in ("prefill", "zipf", "stack", "decode_router"):
             if name != args.workload:
                 r = measure(name, 1 if name == "stack" else max(10, args.steps // 4), args.warmup)
                 extra[name] = summarize_extra(r, peaks, peaks_kind)
@@ -361,6 +394,7 @@ def run_gpu(args, rank, world, local_rank):
 
 
 KERNEL_SHARE = {"small_t": (1.0, 1.0), "gate_up": (2 / 3, 2 / 3), "down": (1 / 3, 1 / 3)}
+# (the small-T kernel does the whole layer, the router's share included)
 
 
 def measured_traffic(kernel: str, workload: str):
@@ -476,7 +510,8 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="b200", choices=["b200", "reference"])
-    ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "zipf", "tiny", "stack"])
+    ap.add_argument("--workload", default="decode",
+                    choices=["decode", "prefill", "zipf", "tiny", "stack", *ROUTER_WORKLOADS])
     ap.add_argument("--no-extra", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--regions", type=int, default=5, help="timed regions; the median is reported")
@@ -489,7 +524,7 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
-    wl = synth.WORKLOADS[args.workload]
+    wl = synth.WORKLOADS[ROUTER_WORKLOADS.get(args.workload, args.workload)]
     config = {"workload": f"{wl.name}: T={wl.T} H={wl.H} E={wl.E} top_k={wl.k} I={wl.I} Is={wl.Is}, "
                           f"int4 g64 affine weights, seed {wl.seed}",
               "T": wl.T, "H": wl.H, "E": wl.E, "top_k": wl.k, "I": wl.I, "Is": wl.Is,

@@ -220,6 +220,25 @@ def make_layer(T, H, E, k, I, Is, seed, logit_std=1.0, zipf_s=None,
                        packed, scales, biases, shp, shs, shb)
 
 
+def draw_router(rng, E: int, H: int, logit_std: float) -> np.ndarray:
+    """Router weight [E, H] as bf16 bit patterns, N(0, 1) * logit_std / sqrt(H):
+    with x ~ N(0, 1) the router scores have standard deviation ~logit_std."""
+    w = rng.standard_normal((E, H), dtype=np.float32) * np.float32(logit_std / math.sqrt(H))
+    return bf16_rne(w)
+
+
+def make_router_layer(T, H, E, k, I, Is, seed, logit_std=2.0):
+    """A layer whose logits come from a router weight instead of being given:
+    draws x, then the router weight [E, H], then the experts (``logits`` is
+    left empty: the method computes it). Returns (LayerInputs, router_w)."""
+    rng = np.random.default_rng(seed)
+    x = bf16_rne(rng.standard_normal((T, H), dtype=np.float32))
+    router_w = draw_router(rng, E, H, logit_std)
+    packed, scales, biases, shp, shs, shb = draw_weights(rng, H, E, I, Is)
+    inp = LayerInputs(T, H, E, k, I, Is, x, np.zeros((T, E), np.float32), packed, scales, biases, shp, shs, shb)
+    return inp, router_w
+
+
 def make_workload(name: str, T: int | None = None) -> LayerInputs:
     """Inputs of a single-layer workload (``T`` overrides the token count)."""
     w = WORKLOADS[name]

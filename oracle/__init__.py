@@ -54,6 +54,8 @@ def _load():
         lib.oracle_bf16_value.restype = ctypes.c_double
         lib.oracle_code.argtypes = [P, i]
         lib.oracle_code.restype = i
+        lib.oracle_router_logits.argtypes = [i, i, i, P, P, P]
+        lib.oracle_router_logits.restype = None
         lib.oracle_max_threads.argtypes = []
         lib.oracle_max_threads.restype = i
         _lib = lib
@@ -193,3 +195,30 @@ def moe_forward_by_expert(inp, x: np.ndarray | None = None, logits: np.ndarray |
         o += y[:, k]  # shared expert, weight 1
         out[c0:c1] = o
     return out
+
+
+def router_logits(x: np.ndarray, router_w: np.ndarray) -> np.ndarray:
+    """fp64 router scores [T, E] = x [T, H] . router_w [E, H]^T from bf16 bit patterns."""
+    x, router_w = _c(x, np.uint16), _c(router_w, np.uint16)
+    T, H = x.shape
+    E = router_w.shape[0]
+    assert router_w.shape == (E, H)
+    out = np.empty((T, E), np.float64)
+    _load().oracle_router_logits(T, E, H, _ptr(x), _ptr(router_w), _ptr(out))
+    return out
+
+
+def router_logits_f32(x: np.ndarray, router_w: np.ndarray) -> np.ndarray:
+    """The router scores rounded once to float32, the precision in which the
+    top-k selection compares them (the layer's routing takes float32 logits)."""
+    return router_logits(x, router_w).astype(np.float32)
+
+
+def moe_forward_router(inp, router_w: np.ndarray, x: np.ndarray | None = None, by_expert: bool = False):
+    """The layer with its router: logits = float32(x . router_w^T), then the
+    layer of ``moe_forward`` (or of ``moe_forward_by_expert``) on those logits."""
+    x = _c(inp.x if x is None else x, np.uint16)
+    logits = router_logits_f32(x, router_w)
+    if by_expert:
+        return moe_forward_by_expert(inp, x=x, logits=logits)
+    return moe_forward(inp, x=x, logits=logits)

@@ -161,6 +161,26 @@ int oracle_route(int T, int E, int k, const float *logits, int32_t *ids,
 }
 
 /*
+ * Router scores ("Perplexity open sources Lily...", section "Requirements and
+ * model layout": the router scores every expert of a token):
+ *   logits[t*E + e] = sum_h x[t, h] * w[e, h], in fp64 from the bfloat16 bit
+ * patterns of x [T, H] and the router weight w [E, H] (rows K-contiguous).
+ */
+void oracle_router_logits(int T, int E, int H, const uint16_t *x_bf16, const uint16_t *w_bf16,
+                          double *logits) {
+#ifdef _OPENMP
+#pragma omp parallel for schedule(static)
+#endif
+  for (int t = 0; t < T; ++t)
+    for (int e = 0; e < E; ++e) {
+      double acc = 0.0;
+      for (int h = 0; h < H; ++h)
+        acc += oracle_bf16_value(x_bf16[(size_t)t * H + h]) * oracle_bf16_value(w_bf16[(size_t)e * H + h]);
+      logits[(size_t)t * E + e] = acc;
+    }
+}
+
+/*
  * One SwiGLU expert on one token, fp64 throughout.
  *   words/scales/biases: the expert's three matrices in the packed layout
  *   x [H] input, y [H] output, a [I] scratch.

@@ -337,3 +337,37 @@ def test_by_expert_form_matches_dense_brute_force_tiny():
         Y = np_swiglu_mlp(*np_expert_mats(inp.packed[e], inp.scales[e], inp.biases[e], inp.H, inp.I), X)
         want += R[:, e:e + 1] * Y
     np.testing.assert_allclose(out, want, rtol=1e-10, atol=1e-10 * np.abs(want).max())
+
+
+# ----------------------------------------------------------------------------
+# the router scores (logits = x . W_router^T)
+# ----------------------------------------------------------------------------
+
+def test_router_logits_match_numpy_matmul():
+    inp, w = synth.make_router_layer(6, 512, 32, 4, 128, 128, seed=12)
+    got = oracle.router_logits(inp.x, w)
+    want = synth.bf16_to_f32(inp.x).astype(np.float64) @ synth.bf16_to_f32(w).astype(np.float64).T
+    np.testing.assert_allclose(got, want, rtol=1e-12, atol=1e-12 * np.abs(want).max())
+
+
+def test_router_logits_of_one_hot_input_are_a_weight_column():
+    _, w = synth.make_router_layer(1, 256, 16, 2, 128, 128, seed=13)
+    for h in (0, 63, 64, 255):
+        x = np.zeros((1, 256), np.float32)
+        x[0, h] = 1.0
+        got = oracle.router_logits(synth.bf16_rne(x), w)[0]
+        assert np.array_equal(got, synth.bf16_to_f32(w[:, h]).astype(np.float64))
+
+
+def test_router_logits_scale_exactly_with_a_power_of_two():
+    inp, w = synth.make_router_layer(3, 256, 16, 2, 128, 128, seed=14)
+    x2 = synth.bf16_rne(synth.bf16_to_f32(inp.x) * np.float32(4.0))  # exact in bf16
+    assert np.array_equal(oracle.router_logits(x2, w), 4.0 * oracle.router_logits(inp.x, w))
+
+
+def test_layer_with_router_is_the_layer_on_its_rounded_scores():
+    inp, w = synth.make_router_layer(5, 256, 16, 2, 128, 128, seed=15)
+    logits = oracle.router_logits(inp.x, w).astype(np.float32)
+    assert np.array_equal(oracle.moe_forward_router(inp, w), oracle.moe_forward(inp, logits=logits))
+    assert np.allclose(oracle.moe_forward_router(inp, w, by_expert=True), oracle.moe_forward(inp, logits=logits),
+                       rtol=1e-12, atol=1e-12)
