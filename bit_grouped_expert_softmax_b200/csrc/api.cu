@@ -99,6 +99,14 @@ struct moe_plan_s {
   uint16_t *out_stage;
   int64_t max_gu, max_dn;
   bool test_fault_armed = false;  // MOE_FLAG_TEST_WAIT_TIMEOUT: the next small-T launch carries the fault
+  // moe_forward_host: the copies and the layer of a call that repeats with the
+  // same pinned host buffers, weights and T, captured once and replayed
+  static constexpr int kHostKey = 10;
+  const void *host_key[kHostKey] = {};  // the last call's arguments (T as the last entry)
+  const void *graph_key[kHostKey] = {};
+  cudaGraphExec_t host_graph = nullptr;
+  cudaStream_t capture_stream = nullptr;
+  bool graph_failed = false;            // capture was refused for graph_key: stay eager for it
   // per-kernel timing (moe_profile_enable / moe_profile_read)
   std::vector<cudaEvent_t> prof_events;  // 2 per recorded launch
   std::vector<int> prof_kind;
@@ -182,7 +190,7 @@ moe_status enqueue_routing(moe_plan_s *p, int T, const float *logits, const uint
                       p->wts, p->chunk),
              "route_topk launch");
   }
-  RouteScanArgs sa;
+  RouteScanArgs sa{};
   sa.T = T; sa.E = p->E; sa.k = p->k; sa.H = p->H; sa.I = p->I; sa.Is = p->Is; sa.nchunk = nchunk;
   sa.chunk_cnt = p->chunk; sa.offsets = p->offsets;
   sa.gu_items = p->gu_items; sa.max_gu = static_cast<int>(p->max_gu);
@@ -193,7 +201,7 @@ moe_status enqueue_routing(moe_plan_s *p, int T, const float *logits, const uint
     MOE_CUDA(launch_k(route_scan_kernel, dim3(static_cast<int>(cdiv(p->E, 8))), dim3(256), 0, s, pdl(p), sa),
              "route_scan launch");
   }
-  RouteScatterArgs ca;
+  RouteScatterArgs ca{};
   ca.T = T; ca.E = p->E; ca.k = p->k; ca.H = p->H;
   ca.ids = p->ids; ca.chunk_base = p->chunk; ca.offsets = p->offsets; ca.perm = p->perm; ca.inv = p->inv;
   ca.x = x; ca.xt = p->xt; ca.xexp = p->xexp; ca.status = p->status;
@@ -212,7 +220,7 @@ moe_status enqueue_routing(moe_plan_s *p, int T, const float *logits, const uint
 // Router scores of T tokens into the plan's workspace (grouped path).
 moe_status enqueue_router(moe_plan_s *p, int T, const uint16_t *x, const uint16_t *router_w, float *logits,
                           cudaStream_t s) {
-  RouterArgs r;
+  RouterArgs r{};
   r.T = T; r.E = p->E; r.H = p->H; r.x = x; r.w = router_w; r.logits = logits; r.status = p->status;
   ProfScope ps(p, MOE_KERNEL_ROUTER, s);
   MOE_CUDA(launch_router(r, s, pdl(p)), "router launch");
@@ -229,7 +237,7 @@ moe_status enqueue_layer(moe_plan_s *p, int T, const uint16_t *x, const float *l
   if (use_small_t(p, T) || (p->flags & MOE_FLAG_FORCE_SMALL_T)) {
     if (!small_t_fits(T, p->H, p->k, p->I, p->Is, p->num_sms))
       return fail(MOE_ERR_UNSUPPORTED, "small-T path needs T <= %d and a small enough layer", kSmallT);
-    SmallTArgs a;
+    SmallTArgs a{};
     a.T = T; a.E = p->E; a.k = p->k; a.H = p->H; a.I = p->I; a.Is = p->Is;
     a.x = x; a.logits = router_w ? p->router_logits : logits; a.router_w = router_w;
     a.w = w; a.hbuf = p->hsmall; a.sync = p->small_sync;
@@ -252,7 +260,7 @@ moe_status enqueue_layer(moe_plan_s *p, int T, const uint16_t *x, const float *l
   }
   moe_status st = enqueue_routing(p, T, logits, x, s);
   if (st != MOE_OK) return st;
-  GemmArgs g;
+  GemmArgs g{};
   g.T = T; g.E = p->E; g.k = p->k; g.H = p->H; g.I = p->I; g.Is = p->Is; g.R = T * p->k;
   g.w = w; g.xt = p->xt; g.h = p->h;
   g.h_shared_off = static_cast<int64_t>(p->T_max) * p->k * p->I;
@@ -276,7 +284,7 @@ moe_status enqueue_layer(moe_plan_s *p, int T, const uint16_t *x, const float *l
     ProfScope ps(p, MOE_KERNEL_DOWN, s);
     MOE_CUDA(launch_gemm_down(g, p->num_sms, s, pdl(p)), "down GEMM launch");
   }
-  CombineArgs c;
+  CombineArgs c{};
   c.T = T; c.k = p->k; c.H = p->H; c.R = T * p->k;
   c.inv = p->inv; c.y = p->y; c.xexp = p->xexp; c.residual = residual; c.out = out;
   c.status = p->status; c.debug = (p->flags & MOE_FLAG_DEBUG) ? 1 : 0;
@@ -406,6 +414,8 @@ moe_status moe_plan_destroy(moe_plan_t *plan) {
   cudaError_t err = cudaDeviceSynchronize();
   cudaError_t err2 = cudaFree(plan->ws);
   for (cudaEvent_t e : plan->prof_events) cudaEventDestroy(e);
+  if (plan->host_graph) cudaGraphExecDestroy(plan->host_graph);
+  if (plan->capture_stream) cudaStreamDestroy(plan->capture_stream);
   delete plan;
   if (err != cudaSuccess) return cuda_fail(err, "synchronize before free");
   if (err2 != cudaSuccess) return cuda_fail(err2, "workspace cudaFree");
@@ -481,13 +491,71 @@ moe_status moe_forward_host(moe_plan_t *plan, int T, const void *x_bf16_host, co
   if (st != MOE_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const size_t xb = static_cast<size_t>(T) * plan->H * 2, lb = static_cast<size_t>(T) * plan->E * 4;
-  MOE_CUDA(cudaMemcpyAsync(plan->x_stage, x_bf16_host, xb, cudaMemcpyHostToDevice, s), "copy x to device");
-  MOE_CUDA(cudaMemcpyAsync(plan->logits_stage, router_logits_host, lb, cudaMemcpyHostToDevice, s),
-           "copy logits to device");
   const LayerWeights w = make_weights(packed_w, scales, biases, shared_packed_w, shared_scales, shared_biases);
-  st = enqueue_layer(plan, T, plan->x_stage, plan->logits_stage, w, nullptr, plan->out_stage, s);
+  // the copies and the layer, enqueued on stream q
+  auto enqueue_all = [&](cudaStream_t q) -> moe_status {
+    MOE_CUDA(cudaMemcpyAsync(plan->x_stage, x_bf16_host, xb, cudaMemcpyHostToDevice, q), "copy x to device");
+    MOE_CUDA(cudaMemcpyAsync(plan->logits_stage, router_logits_host, lb, cudaMemcpyHostToDevice, q),
+             "copy logits to device");
+    moe_status s2 = enqueue_layer(plan, T, plan->x_stage, plan->logits_stage, w, nullptr, plan->out_stage, q);
+    if (s2 != MOE_OK) return s2;
+    MOE_CUDA(cudaMemcpyAsync(out_bf16_host, plan->out_stage, xb, cudaMemcpyDeviceToHost, q), "copy out to host");
+    return MOE_OK;
+  };
+  // A call repeating the previous one's arguments (pinned host buffers, no
+  // profiling or test fault pending) is captured into a CUDA graph on a
+  // private stream the second time and replayed from then on: one launch
+  // instead of three copies and the layer's kernels.
+  const void *key[moe_plan_s::kHostKey] = {x_bf16_host, router_logits_host, out_bf16_host, packed_w, scales, biases,
+                                           shared_packed_w, shared_scales, shared_biases,
+                                           reinterpret_cast<const void *>(static_cast<intptr_t>(T))};
+  auto same = [&](const void *const *k2) {
+    for (int i = 0; i < moe_plan_s::kHostKey; ++i)
+      if (k2[i] != key[i]) return false;
+    return true;
+  };
+  auto pinned = [](const void *ptr) {
+    cudaPointerAttributes at;
+    if (cudaPointerGetAttributes(&at, ptr) != cudaSuccess) {
+      cudaGetLastError();
+      return false;
+    }
+    return at.type == cudaMemoryTypeHost;
+  };
+  const bool graphable = plan->prof_kind.empty() && !plan->test_fault_armed && pinned(x_bf16_host) &&
+                         pinned(router_logits_host) && pinned(out_bf16_host);
+  if (graphable && plan->host_graph && same(plan->graph_key)) {
+    MOE_CUDA(cudaGraphLaunch(plan->host_graph, s), "graph launch");
+    MOE_CUDA(cudaStreamSynchronize(s), "stream synchronize");
+    return MOE_OK;
+  }
+  if (graphable && same(plan->host_key) && !(plan->graph_failed && same(plan->graph_key))) {
+    if (!plan->capture_stream) MOE_CUDA(cudaStreamCreateWithFlags(&plan->capture_stream, cudaStreamNonBlocking),
+                                        "capture stream");
+    cudaGraph_t graph = nullptr;
+    cudaGraphExec_t exec = nullptr;
+    MOE_CUDA(cudaStreamBeginCapture(plan->capture_stream, cudaStreamCaptureModeThreadLocal), "begin capture");
+    const moe_status sc = enqueue_all(plan->capture_stream);
+    const cudaError_t ec = cudaStreamEndCapture(plan->capture_stream, &graph);
+    cudaError_t ei = cudaErrorUnknown;
+    if (sc == MOE_OK && ec == cudaSuccess && graph) ei = cudaGraphInstantiate(&exec, graph, 0);
+    if (graph) cudaGraphDestroy(graph);
+    for (int i = 0; i < moe_plan_s::kHostKey; ++i) plan->graph_key[i] = key[i];
+    if (ei == cudaSuccess) {
+      if (plan->host_graph) cudaGraphExecDestroy(plan->host_graph);
+      plan->host_graph = exec;
+      plan->graph_failed = false;
+      MOE_CUDA(cudaGraphLaunch(plan->host_graph, s), "graph launch");
+      MOE_CUDA(cudaStreamSynchronize(s), "stream synchronize");
+      return MOE_OK;
+    }
+    cudaGetLastError();  // the capture was refused: this call and later ones with its key run eagerly
+    g_last_error.clear();
+    plan->graph_failed = true;
+  }
+  for (int i = 0; i < moe_plan_s::kHostKey; ++i) plan->host_key[i] = key[i];
+  st = enqueue_all(s);
   if (st != MOE_OK) return st;
-  MOE_CUDA(cudaMemcpyAsync(out_bf16_host, plan->out_stage, xb, cudaMemcpyDeviceToHost, s), "copy out to host");
   MOE_CUDA(cudaStreamSynchronize(s), "stream synchronize");
   return MOE_OK;
 }

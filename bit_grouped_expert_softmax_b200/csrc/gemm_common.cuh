@@ -1,6 +1,7 @@
-// gemm_common.cuh -- pieces shared by the two grouped expert GEMMs (gate/up and
-// down): bounded warp waits, the teardown drain of in-flight copies, the
-// scale/bias row loads of the dequantisation warps and TMA descriptor set-up.
+// gemm_common.cuh -- pieces shared by the tensor-core kernels (the gate/up and
+// down grouped expert GEMMs, the router): bounded warp waits, the teardown
+// drain of in-flight copies, work-item range checks, the scale/bias row loads
+// and dequantisation of the weight warps, and TMA descriptor set-up.
 #pragma once
 
 #include <cuda.h>
@@ -105,19 +106,6 @@ __device__ __forceinline__ uint16_t pick_bf16(uint2 v, int j) {
   return static_cast<uint16_t>((j & 1) ? w >> 16 : w);
 }
 
-// Dequantise four packed words (32 weights of one row) into 16 fp16 pairs.
-__device__ __forceinline__ void dequant4(uint4 v, __half2 s2, __half2 b2, uint32_t (&d)[16]) {
-  const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-  for (int cw = 0; cw < 4; ++cw) {
-    const uint4 o = dequant_word(wv[cw], s2, b2);
-    d[4 * cw + 0] = o.x;
-    d[4 * cw + 1] = o.y;
-    d[4 * cw + 2] = o.z;
-    d[4 * cw + 3] = o.w;
-  }
-}
-
 // Dequantise two packed words (16 weights of one row) into 8 fp16 pairs.
 __device__ __forceinline__ void dequant2(uint32_t w0, uint32_t w1, __half2 s2, __half2 b2, uint32_t (&d)[8]) {
   const uint4 o0 = dequant_word(w0, s2, b2), o1 = dequant_word(w1, s2, b2);
@@ -129,19 +117,6 @@ __device__ __forceinline__ void dequant2(uint32_t w0, uint32_t w1, __half2 s2, _
   d[5] = o1.y;
   d[6] = o1.z;
   d[7] = o1.w;
-}
-
-// Dequantise eight packed words (one row's K-block of 64 weights) into 32 fp16 pairs.
-__device__ __forceinline__ void dequant8(uint4 v0, uint4 v1, __half2 s2, __half2 b2, uint32_t (&d)[32]) {
-  const uint32_t wv[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
-#pragma unroll
-  for (int cw = 0; cw < 8; ++cw) {
-    const uint4 o = dequant_word(wv[cw], s2, b2);
-    d[4 * cw + 0] = o.x;
-    d[4 * cw + 1] = o.y;
-    d[4 * cw + 2] = o.z;
-    d[4 * cw + 3] = o.w;
-  }
 }
 
 // ---------------------------------------------------------------------------

@@ -15,7 +15,8 @@
 //        of Y staged in shared memory and written out in 16-byte pieces.
 //
 // TMEM: two 128-column accumulator stages (a tile's epilogue overlaps the next
-// tile's main loop) and eight one-K-block weight stages of 32 columns.
+// tile's main loop) and four weight stages of two K-blocks (64 columns) each,
+// so every wait and commit covers 128 elements of K.
 // Warp roles (480 threads): 0 weight TMA, 1 activation TMA, 2 MMA issue,
 // 3-6 epilogue, 7-14 dequantisation. Every wait is bounded.
 #include <algorithm>
@@ -45,11 +46,13 @@ constexpr int kBStageBytes = kStageK * kBAtomBytes;
 constexpr int kSuperK = 4;                     // K-blocks per packed stage
 constexpr int kPkStages = 6;
 constexpr int kPkStageBytes = kTileM * 128;    // 128 weight rows x 32 words
-constexpr int kAStages = 8;                    // TMEM weight stages, one K-block (32 columns) each
+constexpr int kAKB = 2;                        // K-blocks per TMEM weight stage (= per activation stage)
+constexpr int kAStages = 4;                    // TMEM weight stages of two K-blocks (2 x 32 columns) each
+static_assert(kAKB == kStageK, "one weight stage per activation stage");
 constexpr int kAccStages = 2;
 constexpr int kACol0 = kAccStages * kN;
 constexpr int kTmemCols = 512;
-static_assert(kACol0 + kAStages * 32 <= kTmemCols, "TMEM budget");
+static_assert(kACol0 + kAStages * kAKB * 32 <= kTmemCols, "TMEM budget");
 constexpr int kStgBytes = kN * 32 * 2;         // per epilogue warp: kN rows x 32 columns fp16
 
 constexpr int kOffPk = 0;
@@ -227,28 +230,28 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_down_kernel(const GemmArgs a
           break;
         }
         const uint32_t b_addr = smem_u32(sB + sb * kBStageBytes);
-        for (int kh = 0; kh < kStageK; ++kh) {
-          if (!warp_wait(&a_full[sa], pha, abort, a.status, 111)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          if (elect_one()) {
-            const uint32_t a_col = tmem_base + kACol0 + sa * 32;
+        if (!warp_wait(&a_full[sa], pha, abort, a.status, 111)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (elect_one()) {
+#pragma unroll
+          for (int kh = 0; kh < kStageK; ++kh) {
+            const uint32_t a_col = tmem_base + kACol0 + sa * (kAKB * 32) + kh * 32;
 #pragma unroll
             for (int kk = 0; kk < kTileK / 16; ++kk)
               tc_mma_f16_ts(d, a_col + kk * 8, smem_desc_sw128(b_addr + kh * kBAtomBytes + kk * 32), idesc,
                             (ks | kh | kk) != 0 ? 1u : 0u);
-            tc_commit(&a_empty[sa]);
-            if (kh == kStageK - 1) tc_commit(&b_empty[sb]);
           }
-          __syncwarp();
-          if (++sa == kAStages) {
-            sa = 0;
-            pha ^= 1u;
-          }
+          tc_commit(&a_empty[sa]);
+          tc_commit(&b_empty[sb]);
         }
-        if (!ok) break;
+        __syncwarp();
+        if (++sa == kAStages) {
+          sa = 0;
+          pha ^= 1u;
+        }
         if (++sb == kBStages) {
           sb = 0;
           phb ^= 1u;
@@ -341,8 +344,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_down_kernel(const GemmArgs a
     for (int it = first; it < nitems && ok; it = next_item(a, it + gridDim.x, nitems, true, false)) {
       const int nkb = row.K / kTileK;
       SbRow next_row = row;
-      for (int kb = 0; kb < nkb; ++kb) {
-        const int j = kb % kSuperK;
+      for (int kb = 0; kb < nkb; kb += kAKB) {  // two K-blocks per TMEM stage
+        const int j = kb % kSuperK;             // 0 or 2 within the packed stage
         if (j == 0) {
           s_cur = s_nxt;
           b_cur = b_nxt;
@@ -353,12 +356,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_down_kernel(const GemmArgs a
             load_sb4(next_row, 0, s_nxt, b_nxt);
           }
         }
-        if (!warp_wait(&a_empty[sa], pha ^ 1u, abort, a.status, 131)) {
-          ok = false;
-          break;
-        }
-        const __half2 s2 = bf16_to_half2_bcast(pick_bf16(s_cur, j));
-        const __half2 b2 = bf16_to_half2_bcast(pick_bf16(b_cur, j));
+        const __half2 s2a = bf16_to_half2_bcast(pick_bf16(s_cur, j));
+        const __half2 b2a = bf16_to_half2_bcast(pick_bf16(b_cur, j));
+        const __half2 s2b = bf16_to_half2_bcast(pick_bf16(s_cur, j + 1));
+        const __half2 b2b = bf16_to_half2_bcast(pick_bf16(b_cur, j + 1));
         if (j == 0 && !warp_wait(&pk_full[sp], php, abort, a.status, 130)) {
           ok = false;
           break;
@@ -367,7 +368,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_down_kernel(const GemmArgs a
         // 16-byte chunks placed at chunk ^ (r & 7) by the TMA's 128-byte swizzle
         const uint8_t *prow = sPk + sp * kPkStageBytes + r * 128;
         const uint4 v0 = *reinterpret_cast<const uint4 *>(prow + (((2 * j + half) ^ (r & 7)) << 4));
-        if (j == kSuperK - 1 || kb == nkb - 1) {  // words in registers: release the packed stage
+        const uint4 v1 = *reinterpret_cast<const uint4 *>(prow + (((2 * j + 2 + half) ^ (r & 7)) << 4));
+        if (j + kAKB == kSuperK || kb + kAKB >= nkb) {  // words in registers: release the packed stage
           __syncwarp();
           if (lane == 0) mbar_arrive(&pk_empty[sp]);
           if (++sp == kPkStages) {
@@ -375,9 +377,22 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_down_kernel(const GemmArgs a
             php ^= 1u;
           }
         }
-        uint32_t dq[16];
-        dequant4(v0, s2, b2, dq);
-        tmem_st_32x32b_x16(tmem_base + (static_cast<uint32_t>(q * 32) << 16) + kACol0 + sa * 32 + 16 * half, dq);
+        // this warp's half of each of the two K-blocks, in quarters whose
+        // stores overlap the next quarter's arithmetic; one wait at the end
+        const uint32_t ta = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + kACol0 + sa * (kAKB * 32) + 16 * half;
+        uint32_t d8[8];
+        dequant2(v0.x, v0.y, s2a, b2a, d8);
+        if (!warp_wait(&a_empty[sa], pha ^ 1u, abort, a.status, 131)) {
+          ok = false;
+          break;
+        }
+        tmem_st_32x32b_x8(ta, d8);
+        dequant2(v0.z, v0.w, s2a, b2a, d8);
+        tmem_st_32x32b_x8(ta + 8, d8);
+        dequant2(v1.x, v1.y, s2b, b2b, d8);
+        tmem_st_32x32b_x8(ta + 32, d8);
+        dequant2(v1.z, v1.w, s2b, b2b, d8);
+        tmem_st_32x32b_x8(ta + 40, d8);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();

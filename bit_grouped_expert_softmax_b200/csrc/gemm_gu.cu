@@ -12,7 +12,8 @@
 // 128 rows of W_gate and of W_up are dequantised into two A operands that
 // share one activation tile, so each activation byte brought on chip feeds 256
 // weight rows. A single accumulator stage holds gate and up (2 x 128 TMEM
-// columns); four one-K-block weight stages (4 x 64 columns) fill the rest.
+// columns); two weight stages of two K-blocks each (2 x 128 columns) fill the
+// rest, so every wait and commit covers 128 elements of K.
 //
 //   TMA: packed int4 rows (a gate box and an up box, 128-byte swizzle) and
 //        fp16 activation rows (32-row boxes)
@@ -54,8 +55,10 @@ constexpr int kPkStages = 3;
 constexpr int kPkTileBytes = kRows * 128;      // one matrix: kRows rows x 32 words
 constexpr int kPkStageBytes = 2 * kPkTileBytes;
 constexpr int kAccCols = kN;                   // fp32 accumulator columns per matrix
-constexpr int kAStages = 4;                    // TMEM weight stages, one K-block of both matrices each
-constexpr int kAStageCols = 2 * 32;
+constexpr int kAKB = 2;                        // K-blocks per TMEM weight stage (= per activation stage)
+constexpr int kAStages = 2;                    // TMEM weight stages: [K-block 0: gate, up | K-block 1: gate, up]
+constexpr int kAStageCols = kAKB * 2 * 32;
+static_assert(kAKB == kStageK, "one weight stage per activation stage");
 constexpr int kACol0 = 2 * kAccCols;           // one accumulator stage: gate, then up
 constexpr int kTmemCols = 512;
 static_assert(kRows == 128, "one TMEM lane per weight row");
@@ -227,14 +230,15 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_gate_up_kernel(const GemmArg
           break;
         }
         const uint32_t b_addr = smem_u32(sB + sb * kBStageBytes);
-        for (int kh = 0; kh < kStageK; ++kh) {
-          if (!warp_wait(&a_full[sa], pha, abort, a.status, 211)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          if (elect_one()) {
-            const uint32_t a_col = tmem_base + kACol0 + sa * kAStageCols;
+        if (!warp_wait(&a_full[sa], pha, abort, a.status, 211)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (elect_one()) {
+#pragma unroll
+          for (int kh = 0; kh < kStageK; ++kh) {
+            const uint32_t a_col = tmem_base + kACol0 + sa * kAStageCols + kh * 64;
 #pragma unroll
             for (int kk = 0; kk < kTileK / 16; ++kk) {
               const uint64_t bdesc = smem_desc_sw128(b_addr + kh * kBAtomBytes + kk * 32);
@@ -242,16 +246,15 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_gate_up_kernel(const GemmArg
               tc_mma_f16_ts(tmem_base, a_col + kk * 8, bdesc, idesc, acc);
               tc_mma_f16_ts(tmem_base + kAccCols, a_col + 32 + kk * 8, bdesc, idesc, acc);
             }
-            tc_commit(&a_empty[sa]);
-            if (kh == kStageK - 1) tc_commit(&b_empty[sb]);
           }
-          __syncwarp();
-          if (++sa == kAStages) {
-            sa = 0;
-            pha ^= 1u;
-          }
+          tc_commit(&a_empty[sa]);
+          tc_commit(&b_empty[sb]);
         }
-        if (!ok) break;
+        __syncwarp();
+        if (++sa == kAStages) {
+          sa = 0;
+          pha ^= 1u;
+        }
         if (++sb == kBStages) {
           sb = 0;
           phb ^= 1u;
@@ -346,8 +349,8 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_gate_up_kernel(const GemmArg
     }
     for (int it = first; it < nitems && ok; it = next_item(a, it + gridDim.x, nitems, false, false)) {
       SbRow next_row = row;
-      for (int kb = 0; kb < nkb; ++kb) {
-        const int j = kb % kSuperK;
+      for (int kb = 0; kb < nkb; kb += kAKB) {  // two K-blocks per TMEM stage
+        const int j = kb % kSuperK;             // 0 or 2 within the packed stage
         if (j == 0) {
           s_cur = s_nxt;
           b_cur = b_nxt;
@@ -358,8 +361,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_gate_up_kernel(const GemmArg
             load_sb4(next_row, 0, s_nxt, b_nxt);
           }
         }
-        const __half2 s2 = bf16_to_half2_bcast(pick_bf16(s_cur, j));
-        const __half2 b2 = bf16_to_half2_bcast(pick_bf16(b_cur, j));
+        const __half2 s2a = bf16_to_half2_bcast(pick_bf16(s_cur, j));
+        const __half2 b2a = bf16_to_half2_bcast(pick_bf16(b_cur, j));
+        const __half2 s2b = bf16_to_half2_bcast(pick_bf16(s_cur, j + 1));
+        const __half2 b2b = bf16_to_half2_bcast(pick_bf16(b_cur, j + 1));
         if (j == 0 && !warp_wait(&pk_full[sp], php, abort, a.status, 230)) {
           ok = false;
           break;
@@ -369,7 +374,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_gate_up_kernel(const GemmArg
         const uint8_t *prow = sPk + sp * kPkStageBytes + m * kPkTileBytes + r * 128;
         const uint4 v0 = *reinterpret_cast<const uint4 *>(prow + (((2 * j) ^ (r & 7)) << 4));
         const uint4 v1 = *reinterpret_cast<const uint4 *>(prow + (((2 * j + 1) ^ (r & 7)) << 4));
-        if (j == kSuperK - 1 || kb == nkb - 1) {  // words in registers: release the packed stage
+        const uint4 v2 = *reinterpret_cast<const uint4 *>(prow + (((2 * j + 2) ^ (r & 7)) << 4));
+        const uint4 v3 = *reinterpret_cast<const uint4 *>(prow + (((2 * j + 3) ^ (r & 7)) << 4));
+        if (j + kAKB == kSuperK || kb + kAKB >= nkb) {  // words in registers: release the packed stage
           __syncwarp();
           if (lane == 0) mbar_arrive(&pk_empty[sp]);
           if (++sp == kPkStages) {
@@ -377,23 +384,31 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_gate_up_kernel(const GemmArg
             php ^= 1u;
           }
         }
-        // four quarters of the K-block: each quarter's store to tensor memory
-        // is in flight while the next quarter is dequantised; one wait at the
-        // end. The first quarter is computed before the stage is known free.
+        // eight quarters of the two K-blocks: each quarter's store to tensor
+        // memory is in flight while the next quarter is dequantised; one wait
+        // at the end. The first quarter is computed before the stage is known free.
         const uint32_t ta = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + kACol0 + sa * kAStageCols + m * 32;
         uint32_t d8[8];
-        dequant2(v0.x, v0.y, s2, b2, d8);
+        dequant2(v0.x, v0.y, s2a, b2a, d8);
         if (!warp_wait(&a_empty[sa], pha ^ 1u, abort, a.status, 231)) {
           ok = false;
           break;
         }
         tmem_st_32x32b_x8(ta, d8);
-        dequant2(v0.z, v0.w, s2, b2, d8);
+        dequant2(v0.z, v0.w, s2a, b2a, d8);
         tmem_st_32x32b_x8(ta + 8, d8);
-        dequant2(v1.x, v1.y, s2, b2, d8);
+        dequant2(v1.x, v1.y, s2a, b2a, d8);
         tmem_st_32x32b_x8(ta + 16, d8);
-        dequant2(v1.z, v1.w, s2, b2, d8);
+        dequant2(v1.z, v1.w, s2a, b2a, d8);
         tmem_st_32x32b_x8(ta + 24, d8);
+        dequant2(v2.x, v2.y, s2b, b2b, d8);
+        tmem_st_32x32b_x8(ta + 64, d8);
+        dequant2(v2.z, v2.w, s2b, b2b, d8);
+        tmem_st_32x32b_x8(ta + 72, d8);
+        dequant2(v3.x, v3.y, s2b, b2b, d8);
+        tmem_st_32x32b_x8(ta + 80, d8);
+        dequant2(v3.z, v3.w, s2b, b2b, d8);
+        tmem_st_32x32b_x8(ta + 88, d8);
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();

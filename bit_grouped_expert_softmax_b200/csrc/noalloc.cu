@@ -123,10 +123,11 @@ extern "C" moe_status moe_forward_small_t_noalloc(int T, int hidden, int n_exper
   // the array keeps the previous call's contents: clear the counters and the status word
   err = cudaMemsetAsync(slot->ptr, 0, kHeaderBytes, s);
   if (err != cudaSuccess) return fail(MOE_ERR_CUDA, "clearing the static scratch header failed");
-  SmallTArgs a;
+  SmallTArgs a{};  // value-initialised: every field not set below is zero (no router: logits are given)
   a.T = T; a.E = n_experts; a.k = top_k; a.H = hidden; a.I = inter; a.Is = shared_inter;
   a.x = static_cast<const uint16_t *>(x_bf16);
   a.logits = router_logits;
+  a.router_w = nullptr;
   a.w.packed = packed_w;
   a.w.scales = static_cast<const uint16_t *>(scales);
   a.w.biases = static_cast<const uint16_t *>(biases);

@@ -26,9 +26,10 @@
 //            the down rows already in shared memory and weights each token's
 //            result by its routing weight; the warps' results are summed in a
 //            fixed order and rounded once
-//   exit     the last CTA to leave resets the readiness counters for the next
-//            launch on the stream; a CTA that gave up on a wait first waits for
-//            its own copies still in flight
+//   exit     once all its warps are past their last counter poll, a CTA counts
+//            itself out; the CTA that completes the count clears the counters
+//            for the next launch on the stream. A CTA that gave up on a wait
+//            waits for its own copies still in flight before it leaves
 //
 // There is no grid-wide barrier: an expert's down product starts as soon as
 // that expert's h is complete, while other experts' gate/up blocks finish.
@@ -73,6 +74,7 @@ struct SmallTShared {
   int b_iss[4];                        // copies issued into each phase-1 stage
   int d_iss[kMaxU];                    // copies issued into each phase-2 stage
   int nU;
+  int polled;  // warps done reading readiness counters
   int abort;
 };
 
@@ -290,6 +292,7 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs
   if (threadIdx.x == 0) {
     for (int s = 0; s < L.nb + L.nd; ++s) mbar_init(&b_full[s], 1);
     sh.abort = 0;
+    sh.polled = 0;
     sh.ulist[0] = E;
     fence_barrier_init();
     fence_proxy_async_smem();
@@ -439,6 +442,14 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs
   // slice * k + rank of the token's candidate list (key 0: no expert there;
   // it precedes nothing valid and is never among a token's top k, as k <= E).
   const int nsl = (E + 31) / 32;
+  {  // empty entries (key 0) pad each token's list to a multiple of four
+    const int npad = ((nsl * k + 3) & ~3) - nsl * k;
+    if (threadIdx.x < T * npad) {
+      const int t = threadIdx.x / npad, m = nsl * k + threadIdx.x % npad;
+      cand_key[t * kCandPerToken + m] = 0u;
+      cand_id[t * kCandPerToken + m] = 0x7fffffff;
+    }
+  }
   for (int un = warp; un < T * nsl; un += kSTWarps) {
     const int t = un / nsl, sl = un % nsl, e = sl * 32 + lane;
     // coherent load: with the router in this kernel, other CTAs wrote the scores
@@ -471,46 +482,43 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs
   __syncthreads();
 
   // ---- routing, step 2: the token's top k among its slices' candidates --------------------
-  // The token's top k lie among the slices' top k. One lane per candidate:
-  // its rank among all nsl * k candidates of the token (broadcast reads of the
-  // list); the candidate of rank j < k is the token's j-th expert.
+  // The token's top k lie among the slices' top k. One thread per candidate
+  // counts the candidates that precede it (16-byte reads of the token's list,
+  // four independent counts: no long dependent chain); the candidate with
+  // count j < k is the token's j-th expert. The list is padded to a multiple
+  // of four with empty entries (key 0), which precede nothing.
+  const int nc = nsl * k, nc4 = (nc + 3) & ~3;
   {
-    const int nc = nsl * k;
-    const int ngrp = (nc + 31) / 32;
-    for (int un = warp; un < T * ngrp; un += kSTWarps) {
-      const int t = un / ngrp, i = (un % ngrp) * 32 + lane;
+    for (int gi = threadIdx.x; gi < T * nc; gi += kSTThreads) {
+      const int t = gi / nc, i = gi - t * nc;
       const uint32_t *kl = cand_key + t * kCandPerToken;
       const int *il = cand_id + t * kCandPerToken;
-      const uint32_t ck = i < nc ? kl[i] : 0u;
-      const int ci = i < nc ? il[i] : 0x7fffffff;
-      int rank = 0;
-      for (int m = 0; m < nc; ++m) {
-        const uint32_t km = kl[m];
-        rank += (km > ck || (km == ck && il[m] < ci)) ? 1 : 0;
+      const uint32_t ck = kl[i];
+      const int ci = il[i];
+      int r0 = 0, r1 = 0, r2 = 0, r3 = 0;
+#pragma unroll 4
+      for (int m = 0; m < nc4; m += 4) {
+        const uint4 kq = *reinterpret_cast<const uint4 *>(kl + m);
+        const int4 iq = *reinterpret_cast<const int4 *>(il + m);
+        r0 += (kq.x > ck || (kq.x == ck && iq.x < ci)) ? 1 : 0;
+        r1 += (kq.y > ck || (kq.y == ck && iq.y < ci)) ? 1 : 0;
+        r2 += (kq.z > ck || (kq.z == ck && iq.z < ci)) ? 1 : 0;
+        r3 += (kq.w > ck || (kq.w == ck && iq.w < ci)) ? 1 : 0;
       }
-      if (i < nc && ck != 0u && rank < k) {
+      const int rank = r0 + r1 + r2 + r3;
+      if (ck != 0u && rank < k) {
         sh.ids[t][rank] = ci;
         sh.wkey[t][rank] = ck;
+        atomicOr(&sh.bitmap[ci >> 5], 1u << (ci & 31));
       }
     }
   }
   __syncthreads();
-  // renormalised softmax weight of each chosen expert: the softmax over all E
-  // restricted to the chosen k and renormalised is exp(l_j - l_max) over the
-  // sum of those k terms (l_max = the first chosen logit)
-  if (warp < T) {
-    const int t = warp;
-    const float ex = lane < k ? expf(key_float(sh.wkey[t][lane]) - key_float(sh.wkey[t][0])) : 0.f;
-    const float z = warp_sum(ex);
-    if (lane < k) {
-      const int id = sh.ids[t][lane];
-      sh.wt[t][lane] = ex / z;
-      atomicOr(&sh.bitmap[id >> 5], 1u << (id & 31));
-    }
-  }
-  __syncthreads();
-  // distinct experts: u = 1 + the rank of each set bit of the bitmap; u = 0 is shared
+  // in parallel: the distinct experts (warp 0), each token's renormalised
+  // weights (warps 1..T), each (token, slot)'s expert index (warps 9, 10) and
+  // each token's power-of-two scale (warp 11)
   if (warp == 0) {
+    // u = 1 + the rank of each set bit of the bitmap; u = 0 is the shared expert
     int before = 0;
 #pragma unroll
     for (int i = 0; i < kMaxExperts / 32; ++i) {
@@ -518,23 +526,30 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs
       if ((wbits >> lane) & 1u) sh.ulist[1 + before + __popc(wbits & ((1u << lane) - 1u))] = 32 * i + lane;
       before += __popc(wbits);
     }
-    if (lane == 0) {
-      sh.umask[0] = (1u << T) - 1u;
-      for (int t = 0; t < T; ++t) sh.uslot[0][t] = static_cast<int8_t>(k);
-      sh.nU = before + 1;
+    if (lane == 0) sh.nU = before + 1;
+    if (lane < T) sh.uslot[0][lane] = static_cast<int8_t>(k);
+    if (lane == 0) sh.umask[0] = (1u << T) - 1u;
+  } else if (warp <= T) {
+    // the softmax over all E restricted to the chosen k and renormalised is
+    // exp(l_j - l_max) over the sum of those k terms (l_max: the first chosen)
+    const int t = warp - 1;
+    const float ex = lane < k ? expf(key_float(sh.wkey[t][lane]) - key_float(sh.wkey[t][0])) : 0.f;
+    const float z = warp_sum(ex);
+    if (lane < k) sh.wt[t][lane] = ex / z;
+  } else if (warp == 9 || warp == 10) {
+    const int f = (warp - 9) * 32 + lane;  // (token, slot) pairs, T * k <= 128: two passes of 64
+    for (int ff = f; ff < T * k; ff += 64) {
+      const int t = ff / k, j = ff % k, e = sh.ids[t][j];
+      int u = 1 + __popc(sh.bitmap[e >> 5] & ((1u << (e & 31)) - 1u));
+      for (int i = 0; i < (e >> 5); ++i) u += __popc(sh.bitmap[i]);
+      atomicOr(&sh.umask[u], 1u << t);
+      sh.uslot[u][t] = static_cast<int8_t>(j);
     }
-  } else if (threadIdx.x - 32 < T * k) {  // token/slot pairs: mask and slot of their expert
-    const int f = threadIdx.x - 32, t = f / k, j = f % k, e = sh.ids[t][j];
-    int u = 1 + __popc(sh.bitmap[e >> 5] & ((1u << (e & 31)) - 1u));
-    for (int i = 0; i < (e >> 5); ++i) u += __popc(sh.bitmap[i]);
-    atomicOr(&sh.umask[u], 1u << t);
-    sh.uslot[u][t] = static_cast<int8_t>(j);
-  }
-  if (threadIdx.x < kSmallT) {  // per-token power-of-two scale: max |x| in [2, 4) after scaling
-    const float amax = __int_as_float(sh.xexp[threadIdx.x]);
+  } else if (warp == 11 && lane < kSmallT) {  // per-token power-of-two scale: max |x| in [2, 4) after scaling
+    const float amax = __int_as_float(sh.xexp[lane]);
     int ex = 0;
     if (amax > 0.f && amax <= 3.0e38f) ex = min(max(ilogbf(amax) - 1, -100), 100);
-    sh.xexp[threadIdx.x] = ex;
+    sh.xexp[lane] = ex;
   }
   __syncthreads();
   const int nU = sh.nU;
@@ -668,10 +683,37 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs
   }
 
   // ---- down + combine ----------------------------------------------------------------
+  // Each CTA arrives at the exit count once all its warps are done reading
+  // readiness counters (a warp is done after its last poll, or at once if it
+  // has no expert to multiply), so the round trip overlaps the remaining
+  // down products. The CTA that completes the count clears every counter
+  // for the next launch: no CTA reads them any more.
+  auto polls_done = [&]() {  // whole warp, once per warp
+    int last = 0;
+    if (lane == 0) last = atomicAdd(&sh.polled, 1) == kSTWarps - 1;
+    if (__shfl_sync(0xffffffffu, last, 0)) {
+      uint32_t arrived = 0;
+      if (lane == 0)
+        asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;" : "=r"(arrived) : "l"(exit_count) : "memory");
+      if (__shfl_sync(0xffffffffu, arrived, 0) == gridDim.x - 1) {
+        for (int i = lane; i < kSmallTSyncWords; i += 32) a.sync[i] = 0u;
+      }
+    }
+  };
+  if (!has_dblk) polls_done();
   if (has_dblk) {
     const int n0 = blockIdx.x * kRowBlock;
+    // each warp's share of the token staging area, for copies of h rows
+    const size_t h_slice_bytes = (L.red_off / kSTWarps) & ~static_cast<size_t>(15);
     float acc[4] = {0.f, 0.f, 0.f, 0.f};  // rows g, g+8; tokens 2c, 2c+1 (this warp's experts, ascending)
     bool ok2 = __all_sync(0xffffffffu, *abort == 0);
+    bool polled = false;  // this warp's last readiness poll is behind it
+    // pass p (base p * nd) gives warp w the experts base + w, base + w + 16, ...
+    // below min(nU, base + nd): a warp at or past min(nU, nd) has none at all
+    if (warp >= min(nU, L.nd)) {
+      polls_done();
+      polled = true;
+    }
     for (int base = 0; base < nU; base += L.nd) {
       const uint32_t par = (base / L.nd) & 1u;
       if (base > 0) {  // next pass: the ring's stages are free once every warp is done
@@ -689,6 +731,12 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs
         // every row block of expert u has published its h
         ok2 = wait_count(ready + u, static_cast<uint32_t>(Iu / kRowBlock), abort, a.status, 42, u, budget);
         if (!ok2) break;
+        const bool later_in_pass = u + kSTWarps < min(nU, base + L.nd);
+        const bool later_pass = warp < L.nd && base + L.nd + warp < nU;
+        if (!later_in_pass && !later_pass) {  // the warp's last expert: no more polls
+          polls_done();
+          polled = true;
+        }
         const int iw = Iu / 8;  // packed words per down row
         const uint8_t *st = dring + s * L.d_stage;
         const uint32_t *pd = reinterpret_cast<const uint32_t *>(st);
@@ -696,9 +744,29 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs
         const uint16_t *sd = reinterpret_cast<const uint16_t *>(st + kRowBlock * (Imax / 2));
         const uint16_t *bd = sd + kRowBlock * ngd;
         // B fragments: token g's h for this expert (zeros if g is not routed to
-        // it), read from L2 (written by other CTAs of this launch)
+        // it), written by other CTAs of this launch. Where the warp's share of
+        // the token staging area (free once this CTA's gate/up is done) holds
+        // the expert's rows for all T tokens, they are first copied there in
+        // one round trip (cp.async through L2); otherwise read from L2 directly.
         const int jg = (g < T) ? sh.uslot[u][g] : -1;
-        const __half *hrow = hb + (static_cast<size_t>(g) * (k + 1) + (jg < 0 ? 0 : jg)) * Imax;
+        const bool staged = static_cast<size_t>(T) * Iu * 2 <= h_slice_bytes;
+        const __half *hrow;
+        if (staged) {
+          __half *hw = reinterpret_cast<__half *>(dyn + L.x_off + warp * h_slice_bytes);
+          const int cpr = Iu / 8;  // 16-byte chunks per row
+          for (int idx = lane; idx < T * cpr; idx += 32) {
+            const int t = idx / cpr, cc = idx - t * cpr, jt = sh.uslot[u][t];
+            if (jt >= 0)
+              asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(hw + t * Iu + cc * 8)),
+                           "l"(hb + (static_cast<size_t>(t) * (k + 1) + jt) * Imax + cc * 8)
+                           : "memory");
+          }
+          asm volatile("cp.async.wait_all;" ::: "memory");
+          __syncwarp();
+          hrow = hw + (g < T ? g : 0) * Iu;
+        } else {
+          hrow = hb + (static_cast<size_t>(g) * (k + 1) + (jg < 0 ? 0 : jg)) * Imax;
+        }
         float y[4] = {0.f, 0.f, 0.f, 0.f};
         for (int wb = 0; wb < iw; wb += 32) {  // two 16-word blocks per pass: 8 h loads in flight
           uint4 hv[2][4];
@@ -707,8 +775,10 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs
 #pragma unroll
             for (int p = 0; p < 4; ++p) {
               const int w = wb + 16 * b2 + 4 * c + p;
-              hv[b2][p] = (jg >= 0 && w < iw) ? __ldcg(reinterpret_cast<const uint4 *>(hrow + w * 8))
-                                               : make_uint4(0, 0, 0, 0);
+              hv[b2][p] = make_uint4(0, 0, 0, 0);
+              if (jg >= 0 && w < iw)
+                hv[b2][p] = staged ? *reinterpret_cast<const uint4 *>(hrow + w * 8)
+                                   : __ldcg(reinterpret_cast<const uint4 *>(hrow + w * 8));
             }
 #pragma unroll
           for (int b2 = 0; b2 < 2; ++b2) {
@@ -741,6 +811,7 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs
         }
       }
     }
+    if (!polled) polls_done();  // a wait gave up before the last poll
     float *rp = red + static_cast<size_t>(threadIdx.x) * 8;
 #pragma unroll
     for (int i = 0; i < 4; ++i) rp[i] = acc[i];
@@ -769,15 +840,6 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs
     if (*abort) {
       drain_ring(b_full, sh.b_iss, L.nb);
       drain_ring(d_full, sh.d_iss, L.nd);
-    }
-    // every CTA has finished reading the counters once all have arrived here:
-    // the last one clears them for the next launch on the stream
-    uint32_t arrived;
-    asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;" : "=r"(arrived) : "l"(exit_count) : "memory");
-    if (arrived == gridDim.x - 1) {
-      for (int u = 0; u < kMaxU; ++u) ready[u] = 0u;
-      *router_count = 0u;
-      *exit_count = 0u;
     }
   }
 }

@@ -190,7 +190,11 @@ moe_status moe_router_logits(moe_plan_t *plan, int T, const void *x_bf16, const 
  * out_bf16_host are host pointers (pinned memory gives asynchronous copies);
  * the weights are device pointers. Copies the inputs into the plan's device
  * staging buffers, runs the layer, copies the output back and waits for the
- * stream, so the host buffers may be reused on return.
+ * stream, so the host buffers may be reused on return. When a call repeats
+ * the previous call's arguments with pinned host buffers (a decode loop), the
+ * plan captures the copies and the layer into a CUDA graph once and replays
+ * it on later such calls (one launch); results are the same. Not while
+ * profiling is enabled.
  */
 moe_status moe_forward_host(moe_plan_t *plan, int T, const void *x_bf16_host,
                             const float *router_logits_host, const uint32_t *packed_w,

@@ -172,16 +172,27 @@ def test_deterministic_reruns():
     assert np.array_equal(a, b)
 
 
-def test_forward_host_matches_device_call():
-    inp = workload("tiny")
+@pytest.mark.parametrize("name", ["tiny", "decode"])
+def test_forward_host_matches_device_call(name):
+    """Host buffers: the first call runs eagerly, a repeat of it is captured
+    into a graph, later repeats replay the graph; all equal the device call."""
+    inp = workload(name)
     plan = _plan(inp)
     layer = _layer(inp)
     dev = _forward(plan, inp, layer)
     x = torch.from_numpy(inp.x.view(np.int16)).pin_memory()
     lg = torch.from_numpy(inp.logits).pin_memory()
     out = torch.empty_like(x).pin_memory()
-    api.moe_forward_host(plan.handle, inp.T, x, lg, *layer.args(), out)
-    assert np.array_equal(out.numpy(), dev)
+    for call in range(4):
+        out.fill_(0x7FC0)
+        api.moe_forward_host(plan.handle, inp.T, x, lg, *layer.args(), out)
+        assert np.array_equal(out.numpy(), dev), f"call {call}"
+    plan.status_sync()
+    # pageable buffers take the eager path
+    xp, lp, op = inp.x.copy(), inp.logits.copy(), np.empty_like(inp.x)
+    for call in range(2):
+        api.moe_forward_host(plan.handle, inp.T, xp, lp, *layer.args(), op)
+        assert np.array_equal(op.view(np.int16), dev), f"pageable call {call}"
 
 
 def test_output_canaries_untouched():
