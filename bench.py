@@ -371,7 +371,9 @@ def run_gpu(args, rank, world, local_rank):
         lh = torch.from_numpy(inp.logits).pin_memory()
         oh = torch.empty_like(xh).pin_memory()
         xp, lp, op = xh.data_ptr(), lh.data_ptr(), oh.data_ptr()
-        for i in range(3):
+        # two passes over the weight replicas: the library captures each call's
+        # graph on its second occurrence, so the timed calls replay graphs
+        for i in range(max(3, 2 * n_rep)):
             api.moe_forward_host(plan.handle, inp.T, xp, lp, *rep_ptrs[i % n_rep], op, stream)
         n_e2e = max(50, min(2000, int(0.2 / max(ms_step * 1e-3, 1e-6))))
         torch.cuda.synchronize(dev)

@@ -99,14 +99,22 @@ struct moe_plan_s {
   uint16_t *out_stage;
   int64_t max_gu, max_dn;
   bool test_fault_armed = false;  // MOE_FLAG_TEST_WAIT_TIMEOUT: the next small-T launch carries the fault
-  // moe_forward_host: the copies and the layer of a call that repeats with the
-  // same pinned host buffers, weights and T, captured once and replayed
+  // moe_forward_host: the copies and the layer of a call whose arguments
+  // (pinned host buffers, weights, T) were seen before, captured into a CUDA
+  // graph and replayed; up to kHostGraphs argument sets, the oldest replaced
   static constexpr int kHostKey = 10;
-  const void *host_key[kHostKey] = {};  // the last call's arguments (T as the last entry)
-  const void *graph_key[kHostKey] = {};
-  cudaGraphExec_t host_graph = nullptr;
+  static constexpr int kHostGraphs = 64;
+  struct HostKey {
+    const void *v[kHostKey];
+    bool operator==(const HostKey &o) const { return std::memcmp(v, o.v, sizeof v) == 0; }
+  };
+  struct HostGraph {
+    HostKey key;
+    cudaGraphExec_t exec;  // null: capture was refused, run eagerly
+  };
+  std::vector<HostKey> host_seen;    // argument sets run once eagerly
+  std::vector<HostGraph> host_graphs;
   cudaStream_t capture_stream = nullptr;
-  bool graph_failed = false;            // capture was refused for graph_key: stay eager for it
   // per-kernel timing (moe_profile_enable / moe_profile_read)
   std::vector<cudaEvent_t> prof_events;  // 2 per recorded launch
   std::vector<int> prof_kind;
@@ -250,7 +258,7 @@ moe_status enqueue_layer(moe_plan_s *p, int T, const uint16_t *x, const float *l
       p->test_fault_armed = false;
     }
     ProfScope ps(p, MOE_KERNEL_SMALL_T, s);
-    MOE_CUDA(launch_small_t(a, p->num_sms, s), "small-T kernel launch");
+    MOE_CUDA(launch_small_t(a, p->num_sms, s, pdl(p)), "small-T kernel launch");
     return MOE_OK;
   }
   if (router_w) {
@@ -414,7 +422,8 @@ moe_status moe_plan_destroy(moe_plan_t *plan) {
   cudaError_t err = cudaDeviceSynchronize();
   cudaError_t err2 = cudaFree(plan->ws);
   for (cudaEvent_t e : plan->prof_events) cudaEventDestroy(e);
-  if (plan->host_graph) cudaGraphExecDestroy(plan->host_graph);
+  for (auto &g : plan->host_graphs)
+    if (g.exec) cudaGraphExecDestroy(g.exec);
   if (plan->capture_stream) cudaStreamDestroy(plan->capture_stream);
   delete plan;
   if (err != cudaSuccess) return cuda_fail(err, "synchronize before free");
@@ -502,18 +511,14 @@ moe_status moe_forward_host(moe_plan_t *plan, int T, const void *x_bf16_host, co
     MOE_CUDA(cudaMemcpyAsync(out_bf16_host, plan->out_stage, xb, cudaMemcpyDeviceToHost, q), "copy out to host");
     return MOE_OK;
   };
-  // A call repeating the previous one's arguments (pinned host buffers, no
-  // profiling or test fault pending) is captured into a CUDA graph on a
-  // private stream the second time and replayed from then on: one launch
-  // instead of three copies and the layer's kernels.
-  const void *key[moe_plan_s::kHostKey] = {x_bf16_host, router_logits_host, out_bf16_host, packed_w, scales, biases,
-                                           shared_packed_w, shared_scales, shared_biases,
-                                           reinterpret_cast<const void *>(static_cast<intptr_t>(T))};
-  auto same = [&](const void *const *k2) {
-    for (int i = 0; i < moe_plan_s::kHostKey; ++i)
-      if (k2[i] != key[i]) return false;
-    return true;
-  };
+  // A call whose arguments (pinned host buffers, no profiling or test fault
+  // pending) were seen before is captured into a CUDA graph on a private
+  // stream and replayed from then on: one launch instead of three copies and
+  // the layer's kernels. The first occurrence runs eagerly (it also sets the
+  // kernels' launch attributes, outside any capture).
+  moe_plan_s::HostKey key = {{x_bf16_host, router_logits_host, out_bf16_host, packed_w, scales, biases,
+                              shared_packed_w, shared_scales, shared_biases,
+                              reinterpret_cast<const void *>(static_cast<intptr_t>(T))}};
   auto pinned = [](const void *ptr) {
     cudaPointerAttributes at;
     if (cudaPointerGetAttributes(&at, ptr) != cudaSuccess) {
@@ -524,36 +529,50 @@ moe_status moe_forward_host(moe_plan_t *plan, int T, const void *x_bf16_host, co
   };
   const bool graphable = plan->prof_kind.empty() && !plan->test_fault_armed && pinned(x_bf16_host) &&
                          pinned(router_logits_host) && pinned(out_bf16_host);
-  if (graphable && plan->host_graph && same(plan->graph_key)) {
-    MOE_CUDA(cudaGraphLaunch(plan->host_graph, s), "graph launch");
-    MOE_CUDA(cudaStreamSynchronize(s), "stream synchronize");
-    return MOE_OK;
-  }
-  if (graphable && same(plan->host_key) && !(plan->graph_failed && same(plan->graph_key))) {
-    if (!plan->capture_stream) MOE_CUDA(cudaStreamCreateWithFlags(&plan->capture_stream, cudaStreamNonBlocking),
-                                        "capture stream");
-    cudaGraph_t graph = nullptr;
-    cudaGraphExec_t exec = nullptr;
-    MOE_CUDA(cudaStreamBeginCapture(plan->capture_stream, cudaStreamCaptureModeThreadLocal), "begin capture");
-    const moe_status sc = enqueue_all(plan->capture_stream);
-    const cudaError_t ec = cudaStreamEndCapture(plan->capture_stream, &graph);
-    cudaError_t ei = cudaErrorUnknown;
-    if (sc == MOE_OK && ec == cudaSuccess && graph) ei = cudaGraphInstantiate(&exec, graph, 0);
-    if (graph) cudaGraphDestroy(graph);
-    for (int i = 0; i < moe_plan_s::kHostKey; ++i) plan->graph_key[i] = key[i];
-    if (ei == cudaSuccess) {
-      if (plan->host_graph) cudaGraphExecDestroy(plan->host_graph);
-      plan->host_graph = exec;
-      plan->graph_failed = false;
-      MOE_CUDA(cudaGraphLaunch(plan->host_graph, s), "graph launch");
-      MOE_CUDA(cudaStreamSynchronize(s), "stream synchronize");
-      return MOE_OK;
+  if (graphable) {
+    for (auto &g : plan->host_graphs)
+      if (g.key == key) {
+        if (!g.exec) break;  // refused before: eager
+        MOE_CUDA(cudaGraphLaunch(g.exec, s), "graph launch");
+        MOE_CUDA(cudaStreamSynchronize(s), "stream synchronize");
+        return MOE_OK;
+      }
+    bool seen = false;
+    for (auto &k2 : plan->host_seen) seen = seen || k2 == key;
+    bool known = false;
+    for (auto &g : plan->host_graphs) known = known || g.key == key;
+    if (seen && !known) {
+      if (!plan->capture_stream)
+        MOE_CUDA(cudaStreamCreateWithFlags(&plan->capture_stream, cudaStreamNonBlocking), "capture stream");
+      cudaGraph_t graph = nullptr;
+      cudaGraphExec_t exec = nullptr;
+      MOE_CUDA(cudaStreamBeginCapture(plan->capture_stream, cudaStreamCaptureModeThreadLocal), "begin capture");
+      const moe_status sc = enqueue_all(plan->capture_stream);
+      const cudaError_t ec = cudaStreamEndCapture(plan->capture_stream, &graph);
+      cudaError_t ei = cudaErrorUnknown;
+      if (sc == MOE_OK && ec == cudaSuccess && graph) ei = cudaGraphInstantiate(&exec, graph, 0);
+      if (graph) cudaGraphDestroy(graph);
+      if (ei != cudaSuccess) {  // refused: this argument set runs eagerly from now on
+        cudaGetLastError();
+        g_last_error.clear();
+        exec = nullptr;
+      }
+      if (static_cast<int>(plan->host_graphs.size()) == moe_plan_s::kHostGraphs) {
+        if (plan->host_graphs.front().exec) cudaGraphExecDestroy(plan->host_graphs.front().exec);
+        plan->host_graphs.erase(plan->host_graphs.begin());
+      }
+      plan->host_graphs.push_back({key, exec});
+      if (exec) {
+        MOE_CUDA(cudaGraphLaunch(exec, s), "graph launch");
+        MOE_CUDA(cudaStreamSynchronize(s), "stream synchronize");
+        return MOE_OK;
+      }
+    } else if (!seen) {
+      if (static_cast<int>(plan->host_seen.size()) == moe_plan_s::kHostGraphs)
+        plan->host_seen.erase(plan->host_seen.begin());
+      plan->host_seen.push_back(key);
     }
-    cudaGetLastError();  // the capture was refused: this call and later ones with its key run eagerly
-    g_last_error.clear();
-    plan->graph_failed = true;
   }
-  for (int i = 0; i < moe_plan_s::kHostKey; ++i) plan->host_key[i] = key[i];
   st = enqueue_all(s);
   if (st != MOE_OK) return st;
   MOE_CUDA(cudaStreamSynchronize(s), "stream synchronize");

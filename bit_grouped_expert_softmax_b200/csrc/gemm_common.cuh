@@ -45,6 +45,32 @@ __device__ __forceinline__ void drain_stages(uint64_t *full, uint32_t issued, ui
   }
 }
 
+// The producer side of an N-stage TMA ring, run by one thread: claim() waits
+// (bounded) for the next stage to be free and arms its full barrier with the
+// bytes about to land; advance() steps to the following stage; drain() waits
+// for the copies still in flight, so that a CTA that gave up can exit safely.
+template <int N>
+struct TmaRing {
+  int s = 0;
+  uint32_t ph = 0, issued = 0, issued_ph = 0;
+
+  __device__ __forceinline__ bool claim(uint64_t *empty, uint64_t *full, uint32_t bytes, volatile int *abort,
+                                        DevStatus *st, uint32_t site) {
+    if (!mbar_wait(&empty[s], ph ^ 1u, abort, st, site)) return false;
+    mbar_arrive_expect_tx(&full[s], bytes);
+    issued |= 1u << s;
+    issued_ph = (issued_ph & ~(1u << s)) | (ph << s);
+    return true;
+  }
+  __device__ __forceinline__ void advance() {
+    if (++s == N) {
+      s = 0;
+      ph ^= 1u;
+    }
+  }
+  __device__ __forceinline__ void drain(uint64_t *full) const { drain_stages<N>(full, issued, issued_ph); }
+};
+
 // Whether a work item lies inside the buffers it addresses: its expert, its
 // 128-row weight block and its activation rows (routed rows in [0, R), the
 // shared expert's rows in [R, R + T)); every TMA coordinate of the item

@@ -9,16 +9,19 @@
 // handful of tokens (aioga.com record, paragraph 3), only shrink N.
 //
 //   TMA: packed int4 rows (128-byte swizzle), fp16 h rows (32-row boxes)
-//   8 dequant warps: q*scale + bias -> fp16 -> TMEM (tcgen05.st), the MMA's A
+//   8 dequant warps (two per TMEM lane quarter, four words of each K-block
+//        row each): q*scale + bias -> fp16 -> TMEM (tcgen05.st), the MMA's A
 //   1 thread: tcgen05.mma (A from TMEM, B = h rows from shared memory)
-//   4 epilogue warps: tcgen05.ld, scale by the row's routing weight, fp16 rows
-//        of Y staged in shared memory and written out in 16-byte pieces.
+//   8 epilogue warps (two per lane quarter, alternate 16-row groups):
+//        tcgen05.ld, scale by the row's routing weight, fp16 rows of Y staged
+//        in shared memory and written out in 16-byte pieces.
 //
 // TMEM: two 128-column accumulator stages (a tile's epilogue overlaps the next
 // tile's main loop) and four weight stages of two K-blocks (64 columns) each,
 // so every wait and commit covers 128 elements of K.
-// Warp roles (480 threads): 0 weight TMA, 1 activation TMA, 2 MMA issue,
-// 3-6 epilogue, 7-14 dequantisation. Every wait is bounded.
+// Warp roles (640 threads): 0 weight TMA, 1 activation TMA, 2 MMA issue,
+// 4-11 epilogue, 12-19 dequantisation (warp 3 idle, so that every role's warps
+// see the tensor-memory lane quarter warp % 4). Every wait is bounded.
 #include <algorithm>
 
 #include "gemm_common.cuh"
@@ -30,13 +33,19 @@ namespace {
 using namespace sm100;
 using namespace gemm;
 
-constexpr int kThreads = 480;
 constexpr int kPkWarp = 0;
 constexpr int kBWarp = 1;
 constexpr int kMmaWarp = 2;
-constexpr int kEpiWarp0 = 3;
-constexpr int kDqWarp0 = 7;
-constexpr int kDqWarps = 8;
+constexpr int kEpiPerQ = 2;                    // epilogue warps per TMEM lane quarter
+constexpr int kDqPerQ = 2;                     // dequantisation warps per lane quarter
+constexpr int kEpiWarp0 = 4;
+constexpr int kEpiWarps = 4 * kEpiPerQ;
+constexpr int kDqWarp0 = kEpiWarp0 + kEpiWarps;
+constexpr int kDqWarps = 4 * kDqPerQ;
+constexpr int kThreads = (kDqWarp0 + kDqWarps) * 32;
+constexpr int kDqWords = 8 / kDqPerQ;          // words of a K-block row per dequantisation warp
+static_assert(kThreads <= 1024, "one CTA");
+static_assert(kDqWords == 2 || kDqWords == 4, "a warp takes 8 or 16 bytes of a K-block row");
 
 constexpr int kN = kTileN;                     // activation rows per tile
 constexpr int kStageK = 2;                     // K-blocks per activation stage
@@ -53,7 +62,8 @@ constexpr int kAccStages = 2;
 constexpr int kACol0 = kAccStages * kN;
 constexpr int kTmemCols = 512;
 static_assert(kACol0 + kAStages * kAKB * 32 <= kTmemCols, "TMEM budget");
-constexpr int kStgBytes = kN * 32 * 2;         // per epilogue warp: kN rows x 32 columns fp16
+static_assert(kEpiWarp0 % 4 == 0 && kDqWarp0 % 4 == 0, "warp w of a role reaches TMEM lane quarter w % 4");
+constexpr int kStgBytes = kN * 32 * 2;         // per lane quarter: kN rows x 32 columns fp16
 
 constexpr int kOffPk = 0;
 constexpr int kOffB = kOffPk + kPkStages * kPkStageBytes;
@@ -111,7 +121,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_down_kernel(const GemmArgs a
     }
     for (int s = 0; s < kAccStages; ++s) {
       mbar_init(&acc_full[s], 1);
-      mbar_init(&acc_empty[s], 4);  // four epilogue warps
+      mbar_init(&acc_empty[s], kEpiWarps);
     }
     mbar_init(mma_done, 1);
     *abort = 0;
@@ -145,8 +155,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_down_kernel(const GemmArgs a
   if (warp == kPkWarp) {
     // ------------------------------------------------ producer: packed weights
     if (lane == 0) {
-      int s = 0;
-      uint32_t ph = 0, issued = 0, issued_ph = 0;
+      TmaRing<kPkStages> ring;
       bool ok = true;
       for (int it = next_item(a, blockIdx.x, nitems, true, true); it < nitems && ok;
            it = next_item(a, it + gridDim.x, nitems, true, true)) {
@@ -156,28 +165,20 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_down_kernel(const GemmArgs a
         // rows of K/8 words: an expert's block is 3H such rows, W_down its last H
         const int wrow = (sh ? 0 : wi.group * 3 * H) + 2 * H + wi.mblk * kTileM;
         const CUtensorMap *mw = sh ? &maps.w_sh : &maps.w;
-        for (int sb = 0; sb < (K / kTileK + kSuperK - 1) / kSuperK; ++sb) {
-          if (!mbar_wait(&pk_empty[s], ph ^ 1u, abort, a.status, 100)) {
+        for (int sb = 0; sb < (K / kTileK + kSuperK - 1) / kSuperK; ++sb, ring.advance()) {
+          if (!ring.claim(pk_empty, pk_full, kPkStageBytes, abort, a.status, 100)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&pk_full[s], kPkStageBytes);
-          issued |= 1u << s;
-          issued_ph = (issued_ph & ~(1u << s)) | (ph << s);
-          tma_load_2d(sPk + s * kPkStageBytes, mw, &pk_full[s], sb * kSuperK * 8, wrow);
-          if (++s == kPkStages) {
-            s = 0;
-            ph ^= 1u;
-          }
+          tma_load_2d(sPk + ring.s * kPkStageBytes, mw, &pk_full[ring.s], sb * kSuperK * 8, wrow);
         }
       }
-      if (!ok) drain_stages<kPkStages>(pk_full, issued, issued_ph);
+      if (!ok) ring.drain(pk_full);
     }
   } else if (warp == kBWarp) {
     // ------------------------------------------------ producer: activation rows
     if (lane == 0) {
-      int s = 0;
-      uint32_t ph = 0, issued = 0, issued_ph = 0;
+      TmaRing<kBStages> ring;
       bool ok = true;
       for (int it = next_item(a, blockIdx.x, nitems, true, false); it < nitems && ok;
            it = next_item(a, it + gridDim.x, nitems, true, false)) {
@@ -187,26 +188,19 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_down_kernel(const GemmArgs a
         const CUtensorMap *mb = sh ? &maps.b_sh : &maps.b;
         const int brow0 = sh ? wi.row0 - a.R : wi.row0;
         const int nb = (wi.nrows + kBRows - 1) / kBRows;
-        for (int ks = 0; ks < K / (kTileK * kStageK); ++ks) {
-          if (!mbar_wait(&b_empty[s], ph ^ 1u, abort, a.status, 101)) {
+        for (int ks = 0; ks < K / (kTileK * kStageK); ++ks, ring.advance()) {
+          if (!ring.claim(b_empty, b_full, kStageK * nb * kBRows * 128, abort, a.status, 101)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&b_full[s], kStageK * nb * kBRows * 128);
-          issued |= 1u << s;
-          issued_ph = (issued_ph & ~(1u << s)) | (ph << s);
 #pragma unroll
           for (int kh = 0; kh < kStageK; ++kh)
             for (int j = 0; j < nb; ++j)
-              tma_load_2d(sB + s * kBStageBytes + kh * kBAtomBytes + j * kBRows * 128, mb, &b_full[s],
+              tma_load_2d(sB + ring.s * kBStageBytes + kh * kBAtomBytes + j * kBRows * 128, mb, &b_full[ring.s],
                           (ks * kStageK + kh) * kTileK, brow0 + j * kBRows);
-          if (++s == kBStages) {
-            s = 0;
-            ph ^= 1u;
-          }
         }
       }
-      if (!ok) drain_stages<kBStages>(b_full, issued, issued_ph);
+      if (!ok) ring.drain(b_full);
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------ MMA issuer (whole warp, one elected lane issues)
@@ -269,17 +263,24 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_down_kernel(const GemmArgs a
       }
     }
     __syncwarp();
+  } else if (warp < kEpiWarp0) {
+    // warp 3: no role
   } else if (warp < kDqWarp0) {
     // ------------------------------------------------ epilogue
+    // The kEpiPerQ warps of lane quarter q take the tile's 16-row groups in
+    // turn: warp `sub` the groups g with g % kEpiPerQ == sub.
     const int q = warp & 3;  // TMEM lane quarter this warp may access
-    // this warp's 32 output columns of the tile's rows, staged as [row][32] fp16
-    __half *stg = reinterpret_cast<__half *>(smem + kOffStg + (warp - kEpiWarp0) * kStgBytes);
+    const int sub = (warp - kEpiWarp0) >> 2;
+    // the quarter's 32 output columns of the tile's rows, staged as [row][32]
+    // fp16; the quarter's warps write disjoint rows
+    __half *stg = reinterpret_cast<__half *>(smem + kOffStg + q * kStgBytes);
     int li = 0;
     for (int it = next_item(a, blockIdx.x, nitems, true, false); it < nitems;
          it = next_item(a, it + gridDim.x, nitems, true, false), ++li) {
       const WorkItem wi = a.items[it];
       const int st = li % kAccStages;
       const uint32_t acc_ph = (li / kAccStages) & 1;
+      const int ng = (wi.nrows + 15) >> 4;  // 16-row groups of the tile
       // routing weight of each row, lane l of chunk c holding row 32c + l,
       // loaded before the accumulators are ready
       static_assert(kN / 32 == 4, "four 32-row chunks per tile");
@@ -291,44 +292,52 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_down_kernel(const GemmArgs a
       }
       if (!warp_wait(&acc_full[st], acc_ph, abort, a.status, 120)) break;
       tc_fence_after();
+      if (sub >= ng) {  // no group for this warp: the accumulators are not read
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[st]);
+      }
       const uint32_t tq = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + st * kN;
       __half *obase = a.y + static_cast<int64_t>(wi.row0) * H + wi.mblk * kTileM + q * 32;
-      for (int c0 = 0; c0 < wi.nrows; c0 += 32) {
-        const int c = c0 >> 5;
+      for (int g = sub; g < ng; g += kEpiPerQ) {
+        const int c16 = 16 * g;
+        const int c = g >> 1;
         const float wl = c == 0 ? w_l[0] : c == 1 ? w_l[1] : c == 2 ? w_l[2] : w_l[3];
-        uint32_t r0[32];
-        tmem_ld_32x32b_x32(tq + c0, r0);
+        uint32_t r0[16];
+        tmem_ld_32x32b_x16(tq + c16, r0);
         tmem_ld_wait();
-        if (c0 + 32 >= wi.nrows) {  // accumulators fully read: the next tile's MMAs may start
+        if (g + kEpiPerQ >= ng) {  // this warp's last read of the accumulators
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&acc_empty[st]);
         }
 #pragma unroll
-        for (int jj = 0; jj < 32; ++jj) {
-          const float f = __shfl_sync(0xffffffffu, wl, jj);
-          stg[(c0 + jj) * 32 + lane] = __float2half_rn(f * __uint_as_float(r0[jj]));
+        for (int jj = 0; jj < 16; ++jj) {
+          const float f = __shfl_sync(0xffffffffu, wl, 16 * (g & 1) + jj);
+          stg[(c16 + jj) * 32 + lane] = __float2half_rn(f * __uint_as_float(r0[jj]));
         }
       }
       __syncwarp();
-      // write out: 4 chunks of 16 bytes per row, 8 rows per warp instruction
-      for (int j = lane >> 2; j < wi.nrows; j += 8) {
-        const int c = lane & 3;
-        const uint4 v = *reinterpret_cast<const uint4 *>(stg + j * 32 + c * 8);
-        *reinterpret_cast<uint4 *>(obase + static_cast<int64_t>(j) * H + c * 8) = v;
+      // write out this warp's rows: 4 chunks of 16 bytes per row, 8 rows per warp instruction
+      for (int g = sub; g < ng; g += kEpiPerQ) {
+        const int jend = min(16 * g + 16, wi.nrows);
+        for (int j = 16 * g + (lane >> 2); j < jend; j += 8) {
+          const int c = lane & 3;
+          const uint4 v = *reinterpret_cast<const uint4 *>(stg + j * 32 + c * 8);
+          *reinterpret_cast<uint4 *>(obase + static_cast<int64_t>(j) * H + c * 8) = v;
+        }
       }
       __syncwarp();
     }
   } else {
     // ------------------------------------------------ dequantisation
     // Warp w owns TMEM lane quarter w % 4, i.e. weight rows 32*(w%4) + lane; the
-    // two warps of a quarter take four of the eight words of each row and
-    // K-block. The fp16 values go straight to TMEM (tcgen05.st), where the MMA
-    // reads its A operand.
+    // kDqPerQ warps of a quarter take words kDqWords*pw .. kDqWords*pw +
+    // kDqWords - 1 (pw = dw / 4) of each row and K-block. The fp16 values go
+    // straight to TMEM (tcgen05.st), where the MMA reads its A operand.
     const int dw = warp - kDqWarp0;
     const int q = warp & 3;
     const int r = q * 32 + lane;
-    const int half = dw >> 2;  // words 4*half .. 4*half+3 of each K-block
+    const int pw = dw >> 2;
     int sp = 0, sa = 0;
     uint32_t php = 0, pha = 0;
     bool ok = true;
@@ -367,8 +376,22 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_down_kernel(const GemmArgs a
         // row r of the packed stage: 128 bytes = 4 K-blocks of 8 words, in
         // 16-byte chunks placed at chunk ^ (r & 7) by the TMA's 128-byte swizzle
         const uint8_t *prow = sPk + sp * kPkStageBytes + r * 128;
-        const uint4 v0 = *reinterpret_cast<const uint4 *>(prow + (((2 * j + half) ^ (r & 7)) << 4));
-        const uint4 v1 = *reinterpret_cast<const uint4 *>(prow + (((2 * j + 2 + half) ^ (r & 7)) << 4));
+        // this warp's words of K-block j + kk: 4 kDqWords bytes at byte
+        // 4 kDqWords pw of the block's 32, i.e. in chunk 2 (j + kk) + byte / 16
+        constexpr int kBytes = 4 * kDqWords;
+        const int boff = kBytes * pw;
+        uint32_t v[2][kDqWords];
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk) {
+          const uint8_t *src = prow + (((2 * (j + kk) + (boff >> 4)) ^ (r & 7)) << 4) + (boff & 15);
+          if constexpr (kDqWords == 4) {
+            const uint4 t = *reinterpret_cast<const uint4 *>(src);
+            v[kk][0] = t.x, v[kk][1] = t.y, v[kk][2] = t.z, v[kk][3] = t.w;
+          } else {
+            const uint2 t = *reinterpret_cast<const uint2 *>(src);
+            v[kk][0] = t.x, v[kk][1] = t.y;
+          }
+        }
         if (j + kAKB == kSuperK || kb + kAKB >= nkb) {  // words in registers: release the packed stage
           __syncwarp();
           if (lane == 0) mbar_arrive(&pk_empty[sp]);
@@ -377,22 +400,24 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_down_kernel(const GemmArgs a
             php ^= 1u;
           }
         }
-        // this warp's half of each of the two K-blocks, in quarters whose
-        // stores overlap the next quarter's arithmetic; one wait at the end
-        const uint32_t ta = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + kACol0 + sa * (kAKB * 32) + 16 * half;
+        // each pair of words fills 8 columns; a store overlaps the next pair's
+        // arithmetic, the first pair is computed before the stage is known
+        // free; one wait
+        const uint32_t ta =
+            tmem_base + (static_cast<uint32_t>(q * 32) << 16) + kACol0 + sa * (kAKB * 32) + 4 * kDqWords * pw;
         uint32_t d8[8];
-        dequant2(v0.x, v0.y, s2a, b2a, d8);
+        dequant2(v[0][0], v[0][1], s2a, b2a, d8);
         if (!warp_wait(&a_empty[sa], pha ^ 1u, abort, a.status, 131)) {
           ok = false;
           break;
         }
-        tmem_st_32x32b_x8(ta, d8);
-        dequant2(v0.z, v0.w, s2a, b2a, d8);
-        tmem_st_32x32b_x8(ta + 8, d8);
-        dequant2(v1.x, v1.y, s2b, b2b, d8);
-        tmem_st_32x32b_x8(ta + 32, d8);
-        dequant2(v1.z, v1.w, s2b, b2b, d8);
-        tmem_st_32x32b_x8(ta + 40, d8);
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk)
+#pragma unroll
+          for (int p = 0; p < kDqWords / 2; ++p) {
+            if (kk | p) dequant2(v[kk][2 * p], v[kk][2 * p + 1], kk ? s2b : s2a, kk ? b2b : b2a, d8);
+            tmem_st_32x32b_x8(ta + kk * 32 + 8 * p, d8);
+          }
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();

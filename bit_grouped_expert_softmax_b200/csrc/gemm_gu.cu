@@ -17,14 +17,20 @@
 //
 //   TMA: packed int4 rows (a gate box and an up box, 128-byte swizzle) and
 //        fp16 activation rows (32-row boxes)
-//   8 dequant warps (4 gate, 4 up): q*scale + bias -> fp16 -> TMEM (tcgen05.st)
+//   8 dequant warps (one per TMEM lane quarter and matrix): q*scale + bias
+//        -> fp16 -> TMEM (tcgen05.st)
 //   1 thread: tcgen05.mma, two per 16-wide K step (gate, up), B shared
-//   4 epilogue warps: tcgen05.ld of gate and up for the same rows (same TMEM
-//        lanes), h = silu(g) * u, fp16 in the K order the down GEMM's operand
-//        uses, staged in shared memory and written out in 16-byte pieces.
+//   8 epilogue warps (two per lane quarter, alternate 16-token groups):
+//        tcgen05.ld of gate and up for the same rows (same TMEM lanes),
+//        h = silu(g) * u, fp16 in the K order the down GEMM's operand uses,
+//        staged in shared memory and written out in 16-byte pieces.
 //
-// Warp roles (480 threads): 0 weight TMA, 1 activation TMA, 2 MMA issue,
-// 3-6 epilogue, 7-14 dequantisation. Every wait is bounded.
+// Warp roles (640 threads): 0 weight TMA, 1 activation TMA, 2 MMA issue,
+// 4-11 epilogue, 12-19 dequantisation (warp 3 idle, so that every role's warps
+// see the tensor-memory lane quarter warp % 4). The single accumulator stage
+// is the tile's serial step: two epilogue warps per lane quarter empty it
+// sooner than one; more epilogue or dequantisation warps only took issue
+// slots from each other (measured). Every wait is bounded.
 #include <algorithm>
 
 #include "gemm_common.cuh"
@@ -36,13 +42,18 @@ namespace {
 using namespace sm100;
 using namespace gemm;
 
-constexpr int kThreads = 480;
 constexpr int kPkWarp = 0;
 constexpr int kBWarp = 1;
 constexpr int kMmaWarp = 2;
-constexpr int kEpiWarp0 = 3;
-constexpr int kDqWarp0 = 7;
-constexpr int kDqWarps = 8;
+constexpr int kEpiPerQ = 2;                    // epilogue warps per TMEM lane quarter
+constexpr int kDqPerQ = 1;                     // dequantisation warps per lane quarter and matrix
+constexpr int kEpiWarp0 = 4;
+constexpr int kEpiWarps = 4 * kEpiPerQ;
+constexpr int kDqWarp0 = kEpiWarp0 + kEpiWarps;
+constexpr int kDqWarps = 8 * kDqPerQ;
+constexpr int kThreads = (kDqWarp0 + kDqWarps) * 32;
+static_assert(kThreads <= 1024, "one CTA");
+static_assert(kDqPerQ == 1 || kDqPerQ == 2, "a dequantisation warp takes a whole or half a K-block row");
 
 constexpr int kN = kGuTileN;                   // activation rows per tile
 constexpr int kRows = kGuTileM;                // output rows per tile (rows of each of W_gate, W_up)
@@ -62,8 +73,9 @@ static_assert(kAKB == kStageK, "one weight stage per activation stage");
 constexpr int kACol0 = 2 * kAccCols;           // one accumulator stage: gate, then up
 constexpr int kTmemCols = 512;
 static_assert(kRows == 128, "one TMEM lane per weight row");
+static_assert(kEpiWarp0 % 4 == 0 && kDqWarp0 % 4 == 0, "warp w of a role reaches TMEM lane quarter w % 4");
 static_assert(kACol0 + kAStages * kAStageCols <= kTmemCols, "TMEM budget");
-constexpr int kStgBytes = kN * 32 * 2;         // per epilogue warp: kN tokens x 32 columns fp16
+constexpr int kStgBytes = kN * 32 * 2;         // per lane quarter: kN tokens x 32 columns fp16
 
 constexpr int kOffPk = 0;
 constexpr int kOffB = kOffPk + kPkStages * kPkStageBytes;
@@ -120,7 +132,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_gate_up_kernel(const GemmArg
       mbar_init(&a_empty[s], 1);
     }
     mbar_init(acc_full, 1);
-    mbar_init(acc_empty, 4);  // four epilogue warps
+    mbar_init(acc_empty, kEpiWarps);
     mbar_init(mma_done, 1);
     *abort = 0;
     fence_barrier_init();
@@ -151,8 +163,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_gate_up_kernel(const GemmArg
   if (warp == kPkWarp) {
     // ------------------------------------------------ producer: packed weights
     if (lane == 0) {
-      int s = 0;
-      uint32_t ph = 0, issued = 0, issued_ph = 0;
+      TmaRing<kPkStages> ring;
       bool ok = true;
       for (int it = next_item(a, blockIdx.x, nitems, false, true); it < nitems && ok;
            it = next_item(a, it + gridDim.x, nitems, false, true)) {
@@ -162,55 +173,40 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_gate_up_kernel(const GemmArg
         const int row_g = base + wi.mblk * kRows;
         const int row_u = base + (sh ? a.Is : a.I) + wi.mblk * kRows;
         const CUtensorMap *mw = sh ? &maps.w_sh : &maps.w;
-        for (int sb = 0; sb < (nkb + kSuperK - 1) / kSuperK; ++sb) {
-          if (!mbar_wait(&pk_empty[s], ph ^ 1u, abort, a.status, 200)) {
+        for (int sb = 0; sb < (nkb + kSuperK - 1) / kSuperK; ++sb, ring.advance()) {
+          if (!ring.claim(pk_empty, pk_full, kPkStageBytes, abort, a.status, 200)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&pk_full[s], kPkStageBytes);
-          issued |= 1u << s;
-          issued_ph = (issued_ph & ~(1u << s)) | (ph << s);
-          uint8_t *dst = sPk + s * kPkStageBytes;
-          tma_load_2d(dst, mw, &pk_full[s], sb * kSuperK * 8, row_g);
-          tma_load_2d(dst + kPkTileBytes, mw, &pk_full[s], sb * kSuperK * 8, row_u);
-          if (++s == kPkStages) {
-            s = 0;
-            ph ^= 1u;
-          }
+          uint8_t *dst = sPk + ring.s * kPkStageBytes;
+          tma_load_2d(dst, mw, &pk_full[ring.s], sb * kSuperK * 8, row_g);
+          tma_load_2d(dst + kPkTileBytes, mw, &pk_full[ring.s], sb * kSuperK * 8, row_u);
         }
       }
-      if (!ok) drain_stages<kPkStages>(pk_full, issued, issued_ph);
+      if (!ok) ring.drain(pk_full);
     }
   } else if (warp == kBWarp) {
     // ------------------------------------------------ producer: activation rows
     if (lane == 0) {
-      int s = 0;
-      uint32_t ph = 0, issued = 0, issued_ph = 0;
+      TmaRing<kBStages> ring;
       bool ok = true;
       for (int it = next_item(a, blockIdx.x, nitems, false, false); it < nitems && ok;
            it = next_item(a, it + gridDim.x, nitems, false, false)) {
         const WorkItem wi = a.items[it];
         const int nb = (wi.nrows + kBRows - 1) / kBRows;
-        for (int ks = 0; ks < nkb / kStageK; ++ks) {
-          if (!mbar_wait(&b_empty[s], ph ^ 1u, abort, a.status, 201)) {
+        for (int ks = 0; ks < nkb / kStageK; ++ks, ring.advance()) {
+          if (!ring.claim(b_empty, b_full, kStageK * nb * kBRows * 128, abort, a.status, 201)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&b_full[s], kStageK * nb * kBRows * 128);
-          issued |= 1u << s;
-          issued_ph = (issued_ph & ~(1u << s)) | (ph << s);
 #pragma unroll
           for (int kh = 0; kh < kStageK; ++kh)
             for (int j = 0; j < nb; ++j)
-              tma_load_2d(sB + s * kBStageBytes + kh * kBAtomBytes + j * kBRows * 128, &maps.b, &b_full[s],
+              tma_load_2d(sB + ring.s * kBStageBytes + kh * kBAtomBytes + j * kBRows * 128, &maps.b, &b_full[ring.s],
                           (ks * kStageK + kh) * kTileK, wi.row0 + j * kBRows);
-          if (++s == kBStages) {
-            s = 0;
-            ph ^= 1u;
-          }
         }
       }
-      if (!ok) drain_stages<kBStages>(b_full, issued, issued_ph);
+      if (!ok) ring.drain(b_full);
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------ MMA issuer (whole warp, one elected lane issues)
@@ -272,69 +268,92 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_gate_up_kernel(const GemmArg
       }
     }
     __syncwarp();
+  } else if (warp < kEpiWarp0) {
+    // warp 3: no role
   } else if (warp < kDqWarp0) {
     // ------------------------------------------------ epilogue
-    const int q = warp & 3;  // TMEM lane quarter: rows 32q..32q+31 of both matrices
-    // this warp's 32 output columns of the tile's token rows, staged as [token][32] fp16
-    __half *stg = reinterpret_cast<__half *>(smem + kOffStg + (warp - kEpiWarp0) * kStgBytes);
+    // The kEpiPerQ warps of lane quarter q (rows 32q..32q+31 of both matrices)
+    // take the tile's 16-token groups in turn: warp `sub` the groups g with
+    // g % kEpiPerQ == sub, from tensor memory to shared memory to global.
+    const int q = warp & 3;
+    const int sub = (warp - kEpiWarp0) >> 2;
+    // the quarter's 32 output columns of the tile's tokens, staged as [token][32]
+    // fp16; the quarter's warps write disjoint tokens
+    __half *stg = reinterpret_cast<__half *>(smem + kOffStg + q * kStgBytes);
     const int scol = (lane & ~7) + kperm_dst(lane & 7);  // K-permuted order of the down GEMM's operand
     const uint32_t tq = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+    static_assert(kN == 128, "four 32-token exponent registers per lane");
     int li = 0;
     for (int it = blockIdx.x; it < nitems; it += gridDim.x, ++li) {
       const WorkItem wi = a.items[it];
       const bool sh = wi.group == a.E;
+      const int ng = (wi.nrows + 15) >> 4;  // 16-token groups of the tile
+      // exponent of each token's scaling (lane l of register c: token 32c + l),
+      // loaded while the accumulators are still being computed
+      int e_l[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const int jl = 32 * c + lane;
+        e_l[c] = jl < wi.nrows ? a.row_exp[wi.row0 + jl] : 0;
+      }
       if (!warp_wait(acc_full, li & 1, abort, a.status, 220)) break;
       tc_fence_after();
+      if (sub >= ng) {  // no group for this warp: the accumulators are not read
+        __syncwarp();
+        if (lane == 0) mbar_arrive(acc_empty);
+      }
       const int pitch = sh ? a.Is : a.I;
       __half *obase = (sh ? a.h + a.h_shared_off + static_cast<int64_t>(wi.row0 - a.R) * a.Is
                           : a.h + static_cast<int64_t>(wi.row0) * a.I) +
                       wi.mblk * kRows + q * 32;
-      for (int c0 = 0; c0 < wi.nrows; c0 += 32) {
-        const bool last = c0 + 32 >= wi.nrows;
-        // exponent of each token's scaling, one token per lane, broadcast by shuffles
-        const int jl = c0 + lane;
-        const int e_l = jl < wi.nrows ? a.row_exp[wi.row0 + jl] : 0;
-        // two 16-column halves keep the live registers down
+      for (int g = sub; g < ng; g += kEpiPerQ) {
+        const int c16 = 16 * g;
+        uint32_t g16[16], u16[16];
+        tmem_ld_32x32b_x16(tq + c16, g16);
+        tmem_ld_32x32b_x16(tq + kAccCols + c16, u16);
+        tmem_ld_wait();
+        if (g + kEpiPerQ >= ng) {  // this warp's last read of the accumulators
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(acc_empty);
+        }
+        const int ec = g >> 1;
+        const int e_g = ec == 0 ? e_l[0] : ec == 1 ? e_l[1] : ec == 2 ? e_l[2] : e_l[3];
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          uint32_t g16[16], u16[16];
-          tmem_ld_32x32b_x16(tq + c0 + 16 * hh, g16);
-          tmem_ld_32x32b_x16(tq + kAccCols + c0 + 16 * hh, u16);
-          tmem_ld_wait();
-          if (last && hh == 1) {  // accumulators fully read: the next tile's MMAs may start
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(acc_empty);
-          }
-#pragma unroll
-          for (int jj = 0; jj < 16; ++jj) {
-            const int e = __shfl_sync(0xffffffffu, e_l, 16 * hh + jj);
-            // silu(gate) * up with gate = g 2^e, up = u 2^e, result scaled by 2^-2e
-            const float gt = __uint_as_float(g16[jj]) * pow2i(e);
-            const float sg = __fdividef(gt, 1.0f + __expf(-gt));
-            stg[(c0 + 16 * hh + jj) * 32 + scol] = __float2half_rn(sg * pow2i(-e) * __uint_as_float(u16[jj]));
-          }
+        for (int jj = 0; jj < 16; ++jj) {
+          const int e = __shfl_sync(0xffffffffu, e_g, 16 * (g & 1) + jj);
+          // silu(gate) * up with gate = g 2^e, up = u 2^e, result scaled by 2^-2e
+          const float gt = __uint_as_float(g16[jj]) * pow2i(e);
+          const float sg = __fdividef(gt, 1.0f + __expf(-gt));
+          stg[(c16 + jj) * 32 + scol] = __float2half_rn(sg * pow2i(-e) * __uint_as_float(u16[jj]));
         }
       }
       __syncwarp();
-      // write out: 4 chunks of 16 bytes per token row, 8 rows per warp instruction
-      for (int j = lane >> 2; j < wi.nrows; j += 8) {
-        const int c = lane & 3;
-        const uint4 v = *reinterpret_cast<const uint4 *>(stg + j * 32 + c * 8);
-        *reinterpret_cast<uint4 *>(obase + static_cast<int64_t>(j) * pitch + c * 8) = v;
+      // write out this warp's tokens: 4 chunks of 16 bytes per token row, 8 rows per warp instruction
+      for (int g = sub; g < ng; g += kEpiPerQ) {
+        const int jend = min(16 * g + 16, wi.nrows);
+        for (int j = 16 * g + (lane >> 2); j < jend; j += 8) {
+          const int c = lane & 3;
+          const uint4 v = *reinterpret_cast<const uint4 *>(stg + j * 32 + c * 8);
+          *reinterpret_cast<uint4 *>(obase + static_cast<int64_t>(j) * pitch + c * 8) = v;
+        }
       }
       __syncwarp();
     }
   } else {
     // ------------------------------------------------ dequantisation
-    // Warp w owns TMEM lane quarter w % 4, i.e. weight rows 32*(w%4) + lane;
-    // warps 7..10 dequantise W_gate, 11..14 W_up, eight words per row and
-    // K-block. The fp16 values go straight to TMEM (tcgen05.st), where the MMA
-    // reads its A operand.
+    // Warp w owns TMEM lane quarter w % 4, i.e. weight rows 32*(w%4) + lane,
+    // of W_gate ((dw / 4) % 2 == 0) or W_up, and the 16-byte chunks ch of each
+    // K-block with ch % kDqPerQ == dw / 8 (a K-block row is two such chunks).
+    // The fp16 values go straight to TMEM (tcgen05.st), where the MMA reads its
+    // A operand.
+    {
+    constexpr int kCh = 2 / kDqPerQ;  // chunks per K-block row for this warp
     const int dw = warp - kDqWarp0;
     const int q = warp & 3;
     const int r = q * 32 + lane;
-    const int m = dw >> 2;  // 0: gate, 1: up
+    const int m = (dw >> 2) & 1;  // 0: gate, 1: up
+    const int half = dw >> 3;     // 0 unless kDqPerQ == 2
     int sp = 0, sa = 0;
     uint32_t php = 0, pha = 0;
     bool ok = true;
@@ -370,12 +389,15 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_gate_up_kernel(const GemmArg
           break;
         }
         // row r of the packed tile: 128 bytes = 4 K-blocks of 8 words, in
-        // 16-byte chunks placed at chunk ^ (r & 7) by the TMA's 128-byte swizzle
+        // 16-byte chunks placed at chunk ^ (r & 7) by the TMA's 128-byte swizzle;
+        // chunk c of K-block j + kk is 2 (j + kk) + c
         const uint8_t *prow = sPk + sp * kPkStageBytes + m * kPkTileBytes + r * 128;
-        const uint4 v0 = *reinterpret_cast<const uint4 *>(prow + (((2 * j) ^ (r & 7)) << 4));
-        const uint4 v1 = *reinterpret_cast<const uint4 *>(prow + (((2 * j + 1) ^ (r & 7)) << 4));
-        const uint4 v2 = *reinterpret_cast<const uint4 *>(prow + (((2 * j + 2) ^ (r & 7)) << 4));
-        const uint4 v3 = *reinterpret_cast<const uint4 *>(prow + (((2 * j + 3) ^ (r & 7)) << 4));
+        uint4 v[2][kCh];
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk)
+#pragma unroll
+          for (int c = 0; c < kCh; ++c)
+            v[kk][c] = *reinterpret_cast<const uint4 *>(prow + (((2 * (j + kk) + c * kDqPerQ + half) ^ (r & 7)) << 4));
         if (j + kAKB == kSuperK || kb + kAKB >= nkb) {  // words in registers: release the packed stage
           __syncwarp();
           if (lane == 0) mbar_arrive(&pk_empty[sp]);
@@ -384,31 +406,27 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_gate_up_kernel(const GemmArg
             php ^= 1u;
           }
         }
-        // eight quarters of the two K-blocks: each quarter's store to tensor
-        // memory is in flight while the next quarter is dequantised; one wait
-        // at the end. The first quarter is computed before the stage is known free.
+        // pieces of 8 columns whose stores overlap the next piece's
+        // arithmetic; the first is computed before the stage is known free;
+        // one wait. Chunk c of a K-block fills columns 16 c .. 16 c + 15 of
+        // the matrix's 32 in that K-block's 64.
         const uint32_t ta = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + kACol0 + sa * kAStageCols + m * 32;
         uint32_t d8[8];
-        dequant2(v0.x, v0.y, s2a, b2a, d8);
+        dequant2(v[0][0].x, v[0][0].y, s2a, b2a, d8);
         if (!warp_wait(&a_empty[sa], pha ^ 1u, abort, a.status, 231)) {
           ok = false;
           break;
         }
-        tmem_st_32x32b_x8(ta, d8);
-        dequant2(v0.z, v0.w, s2a, b2a, d8);
-        tmem_st_32x32b_x8(ta + 8, d8);
-        dequant2(v1.x, v1.y, s2a, b2a, d8);
-        tmem_st_32x32b_x8(ta + 16, d8);
-        dequant2(v1.z, v1.w, s2a, b2a, d8);
-        tmem_st_32x32b_x8(ta + 24, d8);
-        dequant2(v2.x, v2.y, s2b, b2b, d8);
-        tmem_st_32x32b_x8(ta + 64, d8);
-        dequant2(v2.z, v2.w, s2b, b2b, d8);
-        tmem_st_32x32b_x8(ta + 72, d8);
-        dequant2(v3.x, v3.y, s2b, b2b, d8);
-        tmem_st_32x32b_x8(ta + 80, d8);
-        dequant2(v3.z, v3.w, s2b, b2b, d8);
-        tmem_st_32x32b_x8(ta + 88, d8);
+#pragma unroll
+        for (int kk = 0; kk < 2; ++kk)
+#pragma unroll
+          for (int c = 0; c < kCh; ++c) {
+            const uint32_t tc = ta + kk * 64 + (c * kDqPerQ + half) * 16;
+            if (kk | c) dequant2(v[kk][c].x, v[kk][c].y, kk ? s2b : s2a, kk ? b2b : b2a, d8);
+            tmem_st_32x32b_x8(tc, d8);
+            dequant2(v[kk][c].z, v[kk][c].w, kk ? s2b : s2a, kk ? b2b : b2a, d8);
+            tmem_st_32x32b_x8(tc + 8, d8);
+          }
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
@@ -419,6 +437,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_gate_up_kernel(const GemmArg
         }
       }
       row = next_row;
+    }
     }
   }
 

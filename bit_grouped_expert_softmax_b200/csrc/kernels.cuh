@@ -146,7 +146,7 @@ cudaError_t launch_gemm_gate_up(const GemmArgs &a, int num_sms, cudaStream_t s, 
 cudaError_t launch_gemm_down(const GemmArgs &a, int num_sms, cudaStream_t s, bool pdl);
 cudaError_t launch_combine(const CombineArgs &a, cudaStream_t s, bool pdl);
 cudaError_t launch_router(const RouterArgs &a, cudaStream_t s, bool pdl);
-cudaError_t launch_small_t(const SmallTArgs &a, int num_sms, cudaStream_t s);
+cudaError_t launch_small_t(const SmallTArgs &a, int num_sms, cudaStream_t s, bool pdl);
 int small_t_grid(int num_sms);
 // whether the fused small-T kernel can run this layer (shared memory, grid)
 bool small_t_fits(int T, int H, int k, int I, int Is, int num_sms);

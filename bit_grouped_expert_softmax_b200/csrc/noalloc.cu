@@ -141,7 +141,7 @@ extern "C" moe_status moe_forward_small_t_noalloc(int T, int hidden, int n_exper
   a.out = static_cast<uint16_t *>(out_bf16);
   a.wait_ns = kWaitBudgetNs;
   a.test_fault = 0;
-  err = launch_small_t(a, slot->num_sms, s);
+  err = launch_small_t(a, slot->num_sms, s, false);
   if (err != cudaSuccess) return fail(MOE_ERR_CUDA, "small-T kernel launch failed");
   if (status_out) {
     err = cudaMemcpyAsync(status_out, slot->ptr + kStatusOff, sizeof(DevStatus), cudaMemcpyDeviceToDevice, s);

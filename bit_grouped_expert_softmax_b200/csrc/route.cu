@@ -211,7 +211,9 @@ __global__ void __launch_bounds__(256) route_scatter_kernel(RouteScatterArgs a) 
 // from its max |x| (exact in fp16 unless the row spans more than fp16's
 // range), converted to fp16 and written, in the K-permuted operand order, to
 // the token's k routed rows (positions from the scatter) and its shared-expert
-// row R + t.
+// row R + t. (Gathering the GEMM's operand rows from one compact fp16 row per
+// token instead, by TMA tile::gather4 or by cp.async, made the gate/up GEMM
+// 1.6-2x slower at T = 4096.)
 __global__ void __launch_bounds__(256) gather_kernel(RouteScatterArgs a) {
   pdl_wait();
   pdl_trigger();
@@ -219,36 +221,46 @@ __global__ void __launch_bounds__(256) gather_kernel(RouteScatterArgs a) {
   const int t = blockIdx.x * (blockDim.x >> 5) + warp;
   if (t >= a.T) return;
   const int H = a.H, k = a.k, R = a.T * k;
-  int rows[kMaxTopK];
-#pragma unroll
-  for (int j = 0; j < kMaxTopK; ++j) rows[j] = (j < k) ? a.inv[static_cast<size_t>(t) * k + j] : -1;
+  __shared__ int srows[8][kMaxTopK];  // each warp's token's routed rows
+  int *rows = srows[warp];
+  if (lane < k) rows[lane] = a.inv[static_cast<size_t>(t) * k + lane];
+  __syncwarp();
   const uint4 *src = reinterpret_cast<const uint4 *>(a.x + static_cast<size_t>(t) * H);
   const int nchunk8 = H / 8;
-  float amax = 0.f;
-  for (int c = lane; c < nchunk8; c += 32) {
-    const uint4 v = __ldg(src + c);
+  // the first 256 chunks (H <= 2048: the whole row) are loaded at once and
+  // kept in registers for the conversion; the rest are read twice
+  constexpr int kHeld = 8;
+  uint4 held[kHeld];
+#pragma unroll
+  for (int i = 0; i < kHeld; ++i) {
+    const int c = lane + 32 * i;
+    held[i] = c < nchunk8 ? __ldg(src + c) : make_uint4(0, 0, 0, 0);
+  }
+  auto absmax8 = [](uint4 v, float m) {
     const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      amax = fmaxf(amax, fabsf(__uint_as_float(w4[q] << 16)));
-      amax = fmaxf(amax, fabsf(__uint_as_float(w4[q] & 0xffff0000u)));
+      m = fmaxf(m, fabsf(__uint_as_float(w4[q] << 16)));
+      m = fmaxf(m, fabsf(__uint_as_float(w4[q] & 0xffff0000u)));
     }
-  }
+    return m;
+  };
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < kHeld; ++i) amax = absmax8(held[i], amax);
+  for (int c = lane + 32 * kHeld; c < nchunk8; c += 32) amax = absmax8(__ldg(src + c), amax);
   amax = warp_max(amax);
   int ex = 0;
   if (amax > 0.f && amax <= 3.0e38f) ex = min(max(ilogbf(amax) - 1, -100), 100);  // scaled max in [2, 4)
   const float scale = exp2f(static_cast<float>(-ex));
   if (lane == 0) a.xexp[t] = ex;
   // per-row epilogue factors of the token's k + 1 rows
-#pragma unroll
-  for (int j = 0; j < kMaxTopK; ++j)
-    if (j < k && lane == j && rows[j] >= 0 && rows[j] < R) a.row_exp[rows[j]] = ex;
+  if (lane < k && rows[lane] >= 0 && rows[lane] < R) a.row_exp[rows[lane]] = ex;
   if (lane == 0) {
     a.row_exp[R + t] = ex;
     a.row_w[R + t] = 1.0f;
   }
-  for (int c = lane; c < nchunk8; c += 32) {
-    const uint4 v = __ldg(src + c);
+  auto to_fp16 = [&](uint4 v) {
     const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
     __half hv[8];
 #pragma unroll
@@ -260,15 +272,22 @@ __global__ void __launch_bounds__(256) gather_kernel(RouteScatterArgs a) {
     uint32_t *op = reinterpret_cast<uint32_t *>(&o);
 #pragma unroll
     for (int s = 0; s < 8; s += 2) op[s / 2] = pack_half2(hv[kperm_src(s)], hv[kperm_src(s + 1)]);
-#pragma unroll
-    for (int j = 0; j < kMaxTopK; ++j) {
-      if (j < k) {
-        const int row = rows[j];
-        if (row >= 0 && row < R) reinterpret_cast<uint4 *>(a.xt + static_cast<size_t>(row) * H)[c] = o;
-      }
+    return o;
+  };
+  // each converted chunk goes to the token's k routed rows and its shared row
+  auto put = [&](int c, uint4 o) {
+    for (int j = 0; j < k; ++j) {
+      const int row = rows[j];
+      if (row >= 0 && row < R) reinterpret_cast<uint4 *>(a.xt + static_cast<size_t>(row) * H)[c] = o;
     }
     reinterpret_cast<uint4 *>(a.xt + static_cast<size_t>(R + t) * H)[c] = o;
+  };
+#pragma unroll
+  for (int i = 0; i < kHeld; ++i) {
+    const int c = lane + 32 * i;
+    if (c < nchunk8) put(c, to_fp16(held[i]));
   }
+  for (int c = lane + 32 * kHeld; c < nchunk8; c += 32) put(c, to_fp16(__ldg(src + c)));
 }
 
 }  // namespace moe

@@ -90,23 +90,18 @@ __global__ void __launch_bounds__(kRThreads, 1) router_kernel(const RouterArgs a
   if (warp == 0) {
     // ------------------------------------------------ TMA producer
     if (lane == 0) {
-      uint32_t issued = 0, issued_ph = 0;
+      TmaRing<kRStages> ring;
       bool ok = true;
-      for (int kb = 0; kb < nkb; ++kb) {
-        const int s = kb % kRStages;
-        const uint32_t ph = (kb / kRStages) & 1u;
-        if (!mbar_wait(&empty[s], ph ^ 1u, abort, a.status, 300)) {
+      for (int kb = 0; kb < nkb; ++kb, ring.advance()) {
+        if (!ring.claim(empty, full, kRStageBytes, abort, a.status, 300)) {
           ok = false;
           break;
         }
-        mbar_arrive_expect_tx(&full[s], kRStageBytes);
-        issued |= 1u << s;
-        issued_ph = (issued_ph & ~(1u << s)) | (ph << s);
-        uint8_t *st = smem + s * kRStageBytes;
-        tma_load_2d(st, &maps.x, &full[s], kb * 64, t0);  // rows past T (or E) read as zeros
-        tma_load_2d(st + kRAtom, &maps.w, &full[s], kb * 64, e0);
+        uint8_t *st = smem + ring.s * kRStageBytes;
+        tma_load_2d(st, &maps.x, &full[ring.s], kb * 64, t0);  // rows past T (or E) read as zeros
+        tma_load_2d(st + kRAtom, &maps.w, &full[ring.s], kb * 64, e0);
       }
-      if (!ok) drain_stages<kRStages>(full, issued, issued_ph);
+      if (!ok) ring.drain(full);
     }
   } else if (warp == 1) {
     // ------------------------------------------------ MMA issuer

@@ -376,9 +376,17 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs
   };
 
   // ---- entry: the shared expert's copies need no routing -----------------------------
+  // They read only the weights, so they are issued before the wait for the
+  // kernel ahead on the stream (programmatic dependent launch): x, the
+  // logits, the counters and the scratch are touched only after it.
   const bool shared_first = blockIdx.x < nrb_sh;  // unit 0 is a shared-expert block
   if (warp == 0 && shared_first) issue_b(0);
   if (warp == 1 && has_dblk) issue_d_range(0, 1);  // expert u = 0 is the shared one
+  pdl_wait();
+  // every CTA of this grid is resident once all have passed here, so the next
+  // launch's CTAs, which take SMs only as this grid's leave, cannot keep one
+  // of them waiting
+  pdl_trigger();
 
   // tokens: every thread loads its chunks of x now (kept in registers) so the
   // loads overlap the logits loads of the routing below; a warp's 32 chunks of
@@ -564,7 +572,7 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs
     const int q = (shared_first ? 1 : 0) + warp - 2;
     if (q < min(my_units, L.nb)) issue_b(q);
   }
-  // stage the tokens: fp16 scaled by 2^-e in operand order; rows t >= T are zero
+  // stage the tokens: fp16 scaled by 2^-e in operand order
 #pragma unroll
   for (int i = 0; i < kXPer; ++i) {
     const int idx = threadIdx.x + i * kSTThreads;
@@ -575,9 +583,8 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs
   for (int idx = threadIdx.x + kXPer * kSTThreads; idx < nxc; idx += kSTThreads)
     *reinterpret_cast<uint4 *>(xs + static_cast<size_t>(idx / hw) * (H + kXPad) + (idx % hw) * 8) =
         x_scaled_fp16(__ldg(reinterpret_cast<const uint4 *>(a.x) + idx), sh.xexp[idx / hw]);
-  for (int idx = nxc + threadIdx.x; idx < kSmallT * hw; idx += kSTThreads)
-    *reinterpret_cast<uint4 *>(xs + static_cast<size_t>(idx / hw) * (H + kXPad) + (idx % hw) * 8) =
-        make_uint4(0, 0, 0, 0);
+  // rows t >= T are left as they are: an mma output column depends only on its
+  // own token column, and the columns of rows t >= T are never read
   __syncthreads();
 
   // ---- gate/up ---------------------------------------------------------------------
@@ -587,7 +594,9 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs
   const int ng = H / kGroup;
   for (int r = 0; r < rounds; ++r) {
     const int q = slot_used ? r * units_per_round + slot : my_units;
+    // two accumulator sets per matrix (even and odd words): shorter dependent chains
     float accg[4] = {0.f, 0.f, 0.f, 0.f}, accu[4] = {0.f, 0.f, 0.f, 0.f};
+    float accg2[4] = {0.f, 0.f, 0.f, 0.f}, accu2[4] = {0.f, 0.f, 0.f, 0.f};
     int u = 0, rb = 0, unit = 0;
     if (q < my_units) {
       unit = blockIdx.x + q * gridDim.x;
@@ -629,10 +638,12 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs
             const uint4 xb = *reinterpret_cast<const uint4 *>(xrow + (w0 + p) * 8);
             const uint4 g0 = dequant_word(ag0[p], sg0, bg0), g1 = dequant_word(ag1[p], sg1, bg1);
             const uint4 u0 = dequant_word(au0[p], su0, bu0), u1 = dequant_word(au1[p], su1, bu1);
-            mma16816(accg, g0.x, g1.x, g0.y, g1.y, xb.x, xb.y);
-            mma16816(accg, g0.z, g1.z, g0.w, g1.w, xb.z, xb.w);
-            mma16816(accu, u0.x, u1.x, u0.y, u1.y, xb.x, xb.y);
-            mma16816(accu, u0.z, u1.z, u0.w, u1.w, xb.z, xb.w);
+            float(&ag)[4] = (p & 1) ? accg2 : accg;
+            float(&au)[4] = (p & 1) ? accu2 : accu;
+            mma16816(ag, g0.x, g1.x, g0.y, g1.y, xb.x, xb.y);
+            mma16816(ag, g0.z, g1.z, g0.w, g1.w, xb.z, xb.w);
+            mma16816(au, u0.x, u1.x, u0.y, u1.y, xb.x, xb.y);
+            mma16816(au, u0.z, u1.z, u0.w, u1.w, xb.z, xb.w);
           }
         }
       }
@@ -641,8 +652,8 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs
     float *rp = red + static_cast<size_t>(threadIdx.x) * 8;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      rp[i] = accg[i];
-      rp[4 + i] = accu[i];
+      rp[i] = accg[i] + accg2[i];
+      rp[4 + i] = accu[i] + accu2[i];
     }
     __syncthreads();
     const bool live = __all_sync(0xffffffffu, *abort == 0);  // warp-uniform: the block below syncs the warp
@@ -667,8 +678,8 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs
           hb[(static_cast<size_t>(t) * (k + 1) + j) * Imax + (row & ~7) + kperm_dst(row & 7)] = __float2half_rn(hv);
         }
       }
-      // publish: the block's h values are visible before the count that says so
-      __threadfence();
+      // publish: the warp barrier orders every lane's h stores before lane 0's
+      // release increment, so a reader that acquires the count sees them
       __syncwarp();
       if (lane == 0 && !(a.test_fault && unit == 0))
         asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(ready + u) : "memory");
@@ -767,7 +778,7 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs
         } else {
           hrow = hb + (static_cast<size_t>(g) * (k + 1) + (jg < 0 ? 0 : jg)) * Imax;
         }
-        float y[4] = {0.f, 0.f, 0.f, 0.f};
+        float y[4] = {0.f, 0.f, 0.f, 0.f}, y2[4] = {0.f, 0.f, 0.f, 0.f};  // even / odd words
         for (int wb = 0; wb < iw; wb += 32) {  // two 16-word blocks per pass: 8 h loads in flight
           uint4 hv[2][4];
 #pragma unroll
@@ -794,8 +805,9 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs
 #pragma unroll
             for (int p = 0; p < 4; ++p) {
               const uint4 d0 = dequant_word(ad0[p], s0, b0), d1 = dequant_word(ad1[p], s1, b1);
-              mma16816(y, d0.x, d1.x, d0.y, d1.y, hv[b2][p].x, hv[b2][p].y);
-              mma16816(y, d0.z, d1.z, d0.w, d1.w, hv[b2][p].z, hv[b2][p].w);
+              float(&yy)[4] = (p & 1) ? y2 : y;
+              mma16816(yy, d0.x, d1.x, d0.y, d1.y, hv[b2][p].x, hv[b2][p].y);
+              mma16816(yy, d0.z, d1.z, d0.w, d1.w, hv[b2][p].z, hv[b2][p].w);
             }
           }
         }
@@ -806,7 +818,7 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs
           if (t < T && ((sh.umask[u] >> t) & 1u)) {
             const int j = sh.uslot[u][t];
             const float wgt = (j == k) ? 1.0f : sh.wt[t][j];
-            acc[i] += wgt * ldexpf(y[i], 2 * sh.xexp[t]);
+            acc[i] += wgt * ldexpf(y[i] + y2[i], 2 * sh.xexp[t]);
           }
         }
       }
@@ -844,17 +856,29 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs
   }
 }
 
-cudaError_t launch_small_t(const SmallTArgs &a, int num_sms, cudaStream_t s) {
+cudaError_t launch_small_t(const SmallTArgs &a, int num_sms, cudaStream_t s, bool pdl) {
   const StLayout L = st_layout(a.H, a.I, a.Is, a.T, a.k);
   const size_t smem = L.bytes;
   // the limit is raised to the most any layout takes, once per device
   static std::atomic<uint64_t> smem_set{0};
   cudaError_t err = gemm::ensure_smem_limit(small_t_kernel, static_cast<int>(kStBudget), smem_set);
   if (err != cudaSuccess) return err;
-  SmallTArgs args = a;
-  void *params[] = {&args};
-  return cudaLaunchCooperativeKernel(reinterpret_cast<const void *>(small_t_kernel),
-                                     dim3(small_t_grid(num_sms)), dim3(kSTThreads), params, smem, s);
+  // cooperative: every CTA resident at once (they wait on one another's
+  // readiness counters); with pdl, also allowed to start while the kernel
+  // ahead on the stream finishes
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(small_t_grid(num_sms));
+  cfg.blockDim = dim3(kSTThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 2 : 1;
+  return cudaLaunchKernelEx(&cfg, small_t_kernel, a);
 }
 
 }  // namespace moe

@@ -1,6 +1,6 @@
 """Summarise Nsight Compute output into short markdown tables.
 
-    python -m bit_grouped_expert_softmax_b200.ncu_summary launches <launches.csv> [--skip-prefix at::]
+    python -m bit_grouped_expert_softmax_b200.ncu_summary launches <launches.csv>
     python -m bit_grouped_expert_softmax_b200.ncu_summary report <raw.csv>
     python -m bit_grouped_expert_softmax_b200.ncu_summary record <raw.csv> <kernel-regex> <name> <workload> <summary.md> <source>...
 
@@ -42,7 +42,12 @@ def _short(name: str) -> str:
     return name.strip()
 
 
-def launches(path: str, skip_prefix: tuple[str, ...] = ("at::",)) -> str:
+# torch's own kernels (fills, the spin kernel that holds a stream while the
+# benchmark enqueues its profiled steps) are not the library's
+TORCH_PREFIXES = ("at::", "native::", "cuda::spin_kernel")
+
+
+def launches(path: str, skip_prefix: tuple[str, ...] = TORCH_PREFIXES) -> str:
     rows = _rows(path)
     hdr = next(i for i, r in enumerate(rows) if "Kernel Name" in r)
     h = rows[hdr]

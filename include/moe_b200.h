@@ -90,11 +90,14 @@ enum {
    * moe_status_sync then reports MOE_ERR_DEVICE_TIMEOUT and clears the
    * state, and later calls on the plan run normally. */
   MOE_FLAG_TEST_WAIT_TIMEOUT = 8,
-  /* Launch the grouped path's kernels in plain stream order. By default each
-   * of them goes out with programmatic dependent launch: it may be scheduled
-   * while the kernel before it on the stream finishes, runs its prologue
-   * (barrier set-up, tensor-memory allocation) and waits for that kernel to
-   * complete before it touches global memory. Results are identical. */
+  /* Launch the layer's kernels in plain stream order. By default each of them
+   * goes out with programmatic dependent launch: it may be scheduled while
+   * the kernel before it on the stream finishes, runs its prologue (barrier
+   * set-up, tensor-memory allocation; the small-batch kernel also requests
+   * the shared expert's weights) and waits for that kernel to complete
+   * before it touches any other global memory. Results are identical. A
+   * caller whose kernel right before the layer writes the layer's weights
+   * sets this flag (a copy or memset before it needs nothing). */
   MOE_FLAG_NO_PDL = 16
 };
 
@@ -190,11 +193,12 @@ moe_status moe_router_logits(moe_plan_t *plan, int T, const void *x_bf16, const 
  * out_bf16_host are host pointers (pinned memory gives asynchronous copies);
  * the weights are device pointers. Copies the inputs into the plan's device
  * staging buffers, runs the layer, copies the output back and waits for the
- * stream, so the host buffers may be reused on return. When a call repeats
- * the previous call's arguments with pinned host buffers (a decode loop), the
- * plan captures the copies and the layer into a CUDA graph once and replays
- * it on later such calls (one launch); results are the same. Not while
- * profiling is enabled.
+ * stream, so the host buffers may be reused on return. With pinned host
+ * buffers, a call whose arguments (buffers, weights, T) the plan has seen
+ * before is captured into a CUDA graph and replayed on later such calls (one
+ * launch instead of three copies and the layer's kernels), for up to 64
+ * argument sets (a decode loop over a model's layers); results are the same.
+ * Not while profiling is enabled.
  */
 moe_status moe_forward_host(moe_plan_t *plan, int T, const void *x_bf16_host,
                             const float *router_logits_host, const uint32_t *packed_w,

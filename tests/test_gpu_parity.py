@@ -266,10 +266,13 @@ def test_bounded_wait_runs_out_and_the_plan_recovers():
         check_output(out.cpu().numpy(), oracle.moe_forward(inp), "after the timeout")
 
 
-def test_programmatic_dependent_launch_gives_identical_results():
-    """Three stacked layers of the grouped path, with the default programmatic
-    dependent launch and in plain stream order: bit-identical outputs."""
-    inp = synth.make_layer(300, 512, 32, 4, 256, 384, seed=23, logit_std=1.0)
+@pytest.mark.parametrize("T", [300, 3])
+def test_programmatic_dependent_launch_gives_identical_results(T):
+    """Three stacked layers, with the default programmatic dependent launch and
+    in plain stream order: bit-identical outputs. T = 300 takes the grouped
+    path; T = 3 the small-batch kernel, whose next layer's CTAs request the
+    shared expert's weights before the layer ahead has finished."""
+    inp = synth.make_layer(T, 512, 32, 4, 256, 384, seed=23, logit_std=1.0)
     layer = _layer(inp)
     rng = np.random.default_rng(5)
     logits = np.stack([synth.draw_logits(rng, inp.T, inp.E, inp.k, 1.0, None) for _ in range(3)])
