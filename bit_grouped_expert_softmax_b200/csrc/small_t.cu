@@ -564,11 +564,9 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs
   const int n_units = nrb_sh + (nU - 1) * nrb;
   const int my_units = blockIdx.x < n_units ? (n_units - 1 - blockIdx.x) / gridDim.x + 1 : 0;
   // the requests block their warp while many copies are outstanding, so each
-  // phase-1 unit goes out from its own warp (2, 3, ...) and the routed experts'
-  // down rows from warp 1, all in parallel
-  if (warp == 1) {
-    if (has_dblk) issue_d_range(1, min(nU, L.nd));
-  } else if (warp >= 2) {
+  // phase-1 unit goes out from its own warp (2, 3, ...); the routed experts'
+  // down rows, needed only after gate/up, follow them (below)
+  if (warp >= 2) {
     const int q = (shared_first ? 1 : 0) + warp - 2;
     if (q < min(my_units, L.nb)) issue_b(q);
   }
@@ -586,12 +584,16 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs
   // rows t >= T are left as they are: an mma output column depends only on its
   // own token column, and the columns of rows t >= T are never read
   __syncthreads();
+  // the down rows go out after every gate/up request of this CTA, so the
+  // memory system serves the gate/up rows first
+  if (warp == 1 && has_dblk) issue_d_range(1, min(nU, L.nd));
 
   // ---- gate/up ---------------------------------------------------------------------
   const int slot = warp / L.ks, kq = warp % L.ks;  // unit slot in a round, K slice of this warp
   const int rounds = (my_units + units_per_round - 1) / units_per_round;
   const bool slot_used = slot < units_per_round;  // warps of an unused slot only join the barriers
   const int ng = H / kGroup;
+  const int n_pub = min(L.ks, 4);  // publishing warps per unit (readiness count per unit)
   for (int r = 0; r < rounds; ++r) {
     const int q = slot_used ? r * units_per_round + slot : my_units;
     // two accumulator sets per matrix (even and odd words): shorter dependent chains
@@ -657,24 +659,23 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs
     }
     __syncthreads();
     const bool live = __all_sync(0xffffffffu, *abort == 0);  // warp-uniform: the block below syncs the warp
-    if (q < my_units && kq == 0 && live) {
-      float G[4] = {0.f, 0.f, 0.f, 0.f}, U[4] = {0.f, 0.f, 0.f, 0.f};
-      for (int zz = 0; zz < L.ks; ++zz) {
-        const float *zp = red + static_cast<size_t>((warp + zz) * 32 + lane) * 8;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          G[i] += zp[i];
-          U[i] += zp[4 + i];
-        }
-      }
+    // The unit's first n_pub warps each reduce the C-fragment elements i = kq,
+    // kq + n_pub, ... over the K slices (slice order), store their h and
+    // publish them with their own release increment: a unit counts n_pub.
+    if (q < my_units && kq < n_pub && live) {
       // C fragment: rows g (i = 0, 1) and g + 8 (i = 2, 3), token columns 2c, 2c + 1
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
+      for (int i = kq; i < 4; i += n_pub) {
+        float G = 0.f, U = 0.f;
+        for (int zz = 0; zz < L.ks; ++zz) {
+          const float *zp = red + static_cast<size_t>((warp - kq + zz) * 32 + lane) * 8;
+          G += zp[i];
+          U += zp[4 + i];
+        }
         const int t = 2 * c + (i & 1);
         const int row = rb * kRowBlock + g + (i >> 1) * 8;
         if (t < T && ((sh.umask[u] >> t) & 1u)) {
           const int j = sh.uslot[u][t];
-          const float hv = swiglu_scaled(G[i], U[i], sh.xexp[t]);
+          const float hv = swiglu_scaled(G, U, sh.xexp[t]);
           hb[(static_cast<size_t>(t) * (k + 1) + j) * Imax + (row & ~7) + kperm_dst(row & 7)] = __float2half_rn(hv);
         }
       }
@@ -694,24 +695,29 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs
   }
 
   // ---- down + combine ----------------------------------------------------------------
-  // Each CTA arrives at the exit count once all its warps are done reading
-  // readiness counters (a warp is done after its last poll, or at once if it
-  // has no expert to multiply), so the round trip overlaps the remaining
-  // down products. The CTA that completes the count clears every counter
-  // for the next launch: no CTA reads them any more.
+  // Each CTA adds itself to the exit count (a release increment, nothing to
+  // wait for) once all its warps are done reading readiness counters (a warp
+  // is done after its last poll, or at once if it has no expert to multiply).
+  // The last warp of CTA 0 then waits (bounded, acquire) for the whole grid's
+  // count and clears every counter for the next launch, which no CTA reads
+  // any more: off the critical path when that warp has no expert of its own,
+  // otherwise after its down products.
   auto polls_done = [&]() {  // whole warp, once per warp
     int last = 0;
     if (lane == 0) last = atomicAdd(&sh.polled, 1) == kSTWarps - 1;
-    if (__shfl_sync(0xffffffffu, last, 0)) {
-      uint32_t arrived = 0;
-      if (lane == 0)
-        asm volatile("atom.add.acq_rel.gpu.global.u32 %0, [%1], 1;" : "=r"(arrived) : "l"(exit_count) : "memory");
-      if (__shfl_sync(0xffffffffu, arrived, 0) == gridDim.x - 1) {
-        for (int i = lane; i < kSmallTSyncWords; i += 32) a.sync[i] = 0u;
-      }
+    if (lane == 0 && last) asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(exit_count) : "memory");
+    __syncwarp();
+  };
+  const bool clears = blockIdx.x == 0 && warp == kSTWarps - 1;
+  auto clear_counters = [&]() {  // whole warp (CTA 0's last), after its own polls_done
+    if (wait_count(exit_count, gridDim.x, abort, a.status, 44, 0, budget)) {
+      for (int i = lane; i < kSmallTSyncWords; i += 32) a.sync[i] = 0u;
     }
   };
-  if (!has_dblk) polls_done();
+  if (!has_dblk) {
+    polls_done();
+    if (clears) clear_counters();
+  }
   if (has_dblk) {
     const int n0 = blockIdx.x * kRowBlock;
     // each warp's share of the token staging area, for copies of h rows
@@ -721,9 +727,14 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs
     bool polled = false;  // this warp's last readiness poll is behind it
     // pass p (base p * nd) gives warp w the experts base + w, base + w + 16, ...
     // below min(nU, base + nd): a warp at or past min(nU, nd) has none at all
+    bool cleared = false;
     if (warp >= min(nU, L.nd)) {
       polls_done();
       polled = true;
+      if (clears && nU <= L.nd) {  // one pass: no block barrier ahead that this wait could hold up
+        clear_counters();
+        cleared = true;
+      }
     }
     for (int base = 0; base < nU; base += L.nd) {
       const uint32_t par = (base / L.nd) & 1u;
@@ -739,8 +750,15 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs
         ok2 = __shfl_sync(0xffffffffu, okw, 0) != 0;
         if (!ok2) break;
         const int Iu = u == 0 ? a.Is : a.I;
+        const int iw = Iu / 8;  // packed words per down row
+        const uint8_t *st = dring + s * L.d_stage;
+        const uint32_t *pd = reinterpret_cast<const uint32_t *>(st);
+        const int ngd = Iu / kGroup;
+        const uint16_t *sd = reinterpret_cast<const uint16_t *>(st + kRowBlock * (Imax / 2));
+        const uint16_t *bd = sd + kRowBlock * ngd;
         // every row block of expert u has published its h
-        ok2 = wait_count(ready + u, static_cast<uint32_t>(Iu / kRowBlock), abort, a.status, 42, u, budget);
+        ok2 = wait_count(ready + u, static_cast<uint32_t>(Iu / kRowBlock * min(L.ks, 4)), abort, a.status, 42, u,
+                         budget);
         if (!ok2) break;
         const bool later_in_pass = u + kSTWarps < min(nU, base + L.nd);
         const bool later_pass = warp < L.nd && base + L.nd + warp < nU;
@@ -748,12 +766,6 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs
           polls_done();
           polled = true;
         }
-        const int iw = Iu / 8;  // packed words per down row
-        const uint8_t *st = dring + s * L.d_stage;
-        const uint32_t *pd = reinterpret_cast<const uint32_t *>(st);
-        const int ngd = Iu / kGroup;
-        const uint16_t *sd = reinterpret_cast<const uint16_t *>(st + kRowBlock * (Imax / 2));
-        const uint16_t *bd = sd + kRowBlock * ngd;
         // B fragments: token g's h for this expert (zeros if g is not routed to
         // it), written by other CTAs of this launch. Where the warp's share of
         // the token staging area (free once this CTA's gate/up is done) holds
@@ -793,8 +805,8 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs
             }
 #pragma unroll
           for (int b2 = 0; b2 < 2; ++b2) {
-            const int w0 = wb + 16 * b2 + 4 * c;
             if (wb + 16 * b2 >= iw) break;
+            const int w0 = wb + 16 * b2 + 4 * c;
             const int grp = w0 / 8;
             const __half2 s0 = bf16_to_half2_bcast(sd[g * ngd + grp]), b0 = bf16_to_half2_bcast(bd[g * ngd + grp]);
             const __half2 s1 = bf16_to_half2_bcast(sd[(g + 8) * ngd + grp]),
@@ -824,6 +836,7 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs
       }
     }
     if (!polled) polls_done();  // a wait gave up before the last poll
+    if (clears && !cleared) clear_counters();
     float *rp = red + static_cast<size_t>(threadIdx.x) * 8;
 #pragma unroll
     for (int i = 0; i < 4; ++i) rp[i] = acc[i];
