@@ -57,9 +57,16 @@ bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 int64_t cdiv(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 // Upper bounds of the two work lists for T tokens.
-int64_t max_gu_items(int64_t T, int64_t E, int64_t k, int64_t I, int64_t Is) {
+// Gate/up work items of a batch of T tokens with tiles of `tile` activation rows, at most.
+int64_t max_gu_items(int64_t T, int64_t E, int64_t k, int64_t I, int64_t Is, int64_t tile) {
   const int64_t R = T * k;
-  return (cdiv(R, kGuTileN) + std::min<int64_t>(E, R)) * (I / kGuTileM) + cdiv(T, kGuTileN) * (Is / kGuTileM);
+  return (cdiv(R, tile) + std::min<int64_t>(E, R)) * (I / kGuTileM) + cdiv(T, tile) * (Is / kGuTileM);
+}
+// ... over every batch a plan for T_max tokens may see (each with its own tile size)
+int64_t max_gu_items_plan(int64_t T_max, int64_t E, int64_t k, int64_t I, int64_t Is) {
+  const int64_t t_small = std::min<int64_t>(T_max, kGuTileNSmall * E / k);  // largest T that takes small tiles
+  return std::max(max_gu_items(T_max, E, k, I, Is, gu_tile_rows(T_max, k, E)),
+                  max_gu_items(t_small, E, k, I, Is, kGuTileNSmall));
 }
 int64_t max_dn_items(int64_t T, int64_t E, int64_t k, int64_t H) {
   const int64_t R = T * k;
@@ -201,7 +208,7 @@ moe_status enqueue_routing(moe_plan_s *p, int T, const float *logits, const uint
   RouteScanArgs sa{};
   sa.T = T; sa.E = p->E; sa.k = p->k; sa.H = p->H; sa.I = p->I; sa.Is = p->Is; sa.nchunk = nchunk;
   sa.chunk_cnt = p->chunk; sa.offsets = p->offsets;
-  sa.gu_items = p->gu_items; sa.max_gu = static_cast<int>(p->max_gu);
+  sa.gu_items = p->gu_items; sa.max_gu = static_cast<int>(p->max_gu); sa.gu_tile = gu_tile_rows(T, p->k, p->E);
   sa.dn_items = p->dn_items; sa.max_dn = static_cast<int>(p->max_dn);
   sa.item_counts = p->item_counts; sa.done = p->scan_done; sa.status = p->status;
   {
@@ -280,7 +287,8 @@ moe_status enqueue_layer(moe_plan_s *p, int T, const uint16_t *x, const float *l
   g.hs_rows = p->T_max;
   g.items = p->gu_items;
   g.item_count = p->item_counts;
-  g.max_items = static_cast<int>(max_gu_items(T, p->E, p->k, p->I, p->Is));
+  g.gu_tile = gu_tile_rows(T, p->k, p->E);
+  g.max_items = static_cast<int>(std::min<int64_t>(max_gu_items(T, p->E, p->k, p->I, p->Is, g.gu_tile), p->max_gu));
   {
     ProfScope ps(p, MOE_KERNEL_GATE_UP, s);
     MOE_CUDA(launch_gemm_gate_up(g, p->num_sms, s, pdl(p)), "gate/up GEMM launch");
@@ -339,7 +347,7 @@ moe_status moe_plan(int T_max, int hidden, int n_experts, int top_k, int inter, 
   p->T_max = T_max; p->H = hidden; p->E = n_experts; p->k = top_k; p->I = inter; p->Is = shared_inter;
   p->flags = flags; p->device = dev; p->num_sms = prop.multiProcessorCount;
   p->test_fault_armed = (flags & MOE_FLAG_TEST_WAIT_TIMEOUT) != 0;
-  p->max_gu = max_gu_items(T_max, n_experts, top_k, inter, shared_inter);
+  p->max_gu = max_gu_items_plan(T_max, n_experts, top_k, inter, shared_inter);
   p->max_dn = max_dn_items(T_max, n_experts, top_k, hidden);
   const size_t T = T_max, H = hidden, E = n_experts, k = top_k, I = inter, Is = shared_inter;
   const size_t R = T * k, nchunk = (T + kRouteChunk - 1) / kRouteChunk;

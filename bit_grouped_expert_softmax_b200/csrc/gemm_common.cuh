@@ -80,7 +80,7 @@ __device__ __forceinline__ bool item_in_range(const GemmArgs &a, const WorkItem 
   const bool sh = wi.group == a.E;
   const int mrows = dn ? a.H : (sh ? a.Is : a.I);
   if (wi.mblk < 0 || wi.mblk >= mrows / kTileM) return false;
-  if (wi.nrows < 1 || wi.nrows > kTileN || wi.row0 < 0) return false;
+  if (wi.nrows < 1 || wi.nrows > (dn ? kTileN : a.gu_tile) || wi.row0 < 0) return false;
   const int64_t end = static_cast<int64_t>(wi.row0) + wi.nrows;
   if (sh) return wi.row0 >= a.R && end <= static_cast<int64_t>(a.R) + a.T;
   return end <= a.R;

@@ -25,12 +25,14 @@
 //        h = silu(g) * u, fp16 in the K order the down GEMM's operand uses,
 //        staged in shared memory and written out in 16-byte pieces.
 //
-// Warp roles (640 threads): 0 weight TMA, 1 activation TMA, 2 MMA issue,
-// 4-11 epilogue, 12-19 dequantisation (warp 3 idle, so that every role's warps
-// see the tensor-memory lane quarter warp % 4). The single accumulator stage
-// is the tile's serial step: two epilogue warps per lane quarter empty it
-// sooner than one; more epilogue or dequantisation warps only took issue
-// slots from each other (measured). Every wait is bounded.
+// Warp roles (128-row tiles, 640 threads): 0 weight TMA, 1 activation TMA,
+// 2 MMA issue, 4-11 epilogue, 12-19 dequantisation (warp 3 idle, so that every
+// role's warps see the tensor-memory lane quarter warp % 4); 32-row tiles
+// (small expert groups): 4-7 epilogue, 8-23 dequantisation. The single
+// accumulator stage is the large tile's serial step: two epilogue warps per
+// lane quarter empty it sooner than one; more epilogue or dequantisation
+// warps only took issue slots from each other (measured). Every wait is
+// bounded.
 #include <algorithm>
 
 #include "gemm_common.cuh"
@@ -45,47 +47,59 @@ using namespace gemm;
 constexpr int kPkWarp = 0;
 constexpr int kBWarp = 1;
 constexpr int kMmaWarp = 2;
-constexpr int kEpiPerQ = 2;                    // epilogue warps per TMEM lane quarter
-constexpr int kDqPerQ = 1;                     // dequantisation warps per lane quarter and matrix
 constexpr int kEpiWarp0 = 4;
-constexpr int kEpiWarps = 4 * kEpiPerQ;
-constexpr int kDqWarp0 = kEpiWarp0 + kEpiWarps;
-constexpr int kDqWarps = 8 * kDqPerQ;
-constexpr int kThreads = (kDqWarp0 + kDqWarps) * 32;
-static_assert(kThreads <= 1024, "one CTA");
-static_assert(kDqPerQ == 1 || kDqPerQ == 2, "a dequantisation warp takes a whole or half a K-block row");
 
-constexpr int kN = kGuTileN;                   // activation rows per tile
 constexpr int kRows = kGuTileM;                // output rows per tile (rows of each of W_gate, W_up)
 constexpr int kStageK = 2;                     // K-blocks per activation stage
-constexpr int kBStages = 3;
-constexpr int kBAtomBytes = kN * 128;          // one K-block of kN activation rows
-constexpr int kBStageBytes = kStageK * kBAtomBytes;
 constexpr int kSuperK = 4;                     // K-blocks per packed stage
-constexpr int kPkStages = 3;
 constexpr int kPkTileBytes = kRows * 128;      // one matrix: kRows rows x 32 words
 constexpr int kPkStageBytes = 2 * kPkTileBytes;
-constexpr int kAccCols = kN;                   // fp32 accumulator columns per matrix
 constexpr int kAKB = 2;                        // K-blocks per TMEM weight stage (= per activation stage)
-constexpr int kAStages = 2;                    // TMEM weight stages: [K-block 0: gate, up | K-block 1: gate, up]
-constexpr int kAStageCols = kAKB * 2 * 32;
+constexpr int kAStageCols = kAKB * 2 * 32;     // [K-block 0: gate, up | K-block 1: gate, up]
 static_assert(kAKB == kStageK, "one weight stage per activation stage");
-constexpr int kACol0 = 2 * kAccCols;           // one accumulator stage: gate, then up
 constexpr int kTmemCols = 512;
 static_assert(kRows == 128, "one TMEM lane per weight row");
-static_assert(kEpiWarp0 % 4 == 0 && kDqWarp0 % 4 == 0, "warp w of a role reaches TMEM lane quarter w % 4");
-static_assert(kACol0 + kAStages * kAStageCols <= kTmemCols, "TMEM budget");
-constexpr int kStgBytes = kN * 32 * 2;         // per lane quarter: kN tokens x 32 columns fp16
 
-constexpr int kOffPk = 0;
-constexpr int kOffB = kOffPk + kPkStages * kPkStageBytes;
-constexpr int kOffStg = kOffB + kBStages * kBStageBytes;
-constexpr int kOffBar = kOffStg + 4 * kStgBytes;
-constexpr int kNumBars = 2 * kPkStages + 2 * kBStages + 2 * kAStages + 2 + 1;
-constexpr int kOffMisc = kOffBar + kNumBars * 8;
-constexpr int kSmem = kOffMisc + 64 + 1024;  // + slack for aligning the base
-static_assert(kOffB % 1024 == 0 && kBAtomBytes % 1024 == 0, "128-byte swizzle tiles need 1024-byte alignment");
-static_assert(kSmem <= 227 * 1024, "shared memory budget");
+// Tile shapes. N = 128 activation rows per tile for large groups; N = 32 when
+// the groups are small (a few dozen tokens per expert): the single
+// accumulator stage then takes 64 TMEM columns instead of 256, which leaves
+// room for a third weight stage, so the dequantisation runs two stages ahead
+// of the MMA instead of one; the smaller activation stages allow deeper
+// rings, and with little epilogue work the warps go to dequantisation
+// (16 dequantisation and 4 epilogue warps instead of 8 and 8: measured
+// faster at T = 512).
+template <int N>
+struct GuTile {
+  static constexpr int kEpiPerQ = N == 128 ? 2 : 1;          // epilogue warps per TMEM lane quarter
+  static constexpr int kDqPerQ = N == 128 ? 1 : 2;           // dequantisation warps per lane quarter and matrix
+  static constexpr int kEpiWarps = 4 * kEpiPerQ;
+  static constexpr int kDqWarp0 = kEpiWarp0 + kEpiWarps;
+  static constexpr int kDqWarps = 8 * kDqPerQ;
+  static constexpr int kThreads = (kDqWarp0 + kDqWarps) * 32;
+  static_assert(kThreads <= 1024, "one CTA");
+  static_assert(kDqPerQ == 1 || kDqPerQ == 2, "a dequantisation warp takes a whole or half a K-block row");
+  static_assert(kEpiWarp0 % 4 == 0 && kDqWarp0 % 4 == 0, "warp w of a role reaches TMEM lane quarter w % 4");
+  static constexpr int kN = N;                               // activation rows per tile
+  static constexpr int kBStages = N == 128 ? 3 : 6;
+  static constexpr int kPkStages = N == 128 ? 3 : 4;
+  static constexpr int kAStages = N == 128 ? 2 : 3;          // TMEM weight stages
+  static constexpr int kBAtomBytes = kN * 128;               // one K-block of kN activation rows
+  static constexpr int kBStageBytes = kStageK * kBAtomBytes;
+  static constexpr int kAccCols = kN;                        // fp32 accumulator columns per matrix
+  static constexpr int kACol0 = 2 * kAccCols;                // one accumulator stage: gate, then up
+  static constexpr int kStgBytes = kN * 32 * 2;              // per lane quarter: kN tokens x 32 columns fp16
+  static constexpr int kOffPk = 0;
+  static constexpr int kOffB = kOffPk + kPkStages * kPkStageBytes;
+  static constexpr int kOffStg = kOffB + kBStages * kBStageBytes;
+  static constexpr int kOffBar = kOffStg + 4 * kStgBytes;
+  static constexpr int kNumBars = 2 * kPkStages + 2 * kBStages + 2 * kAStages + 2 + 1;
+  static constexpr int kOffMisc = kOffBar + kNumBars * 8;
+  static constexpr int kSmem = kOffMisc + 64 + 1024;        // + slack for aligning the base
+  static_assert(kN % 32 == 0 && kN <= 128, "whole 32-row activation boxes");
+  static_assert(kACol0 + kAStages * kAStageCols <= kTmemCols, "TMEM budget");
+  static_assert(kOffB % 1024 == 0 && kBAtomBytes % 1024 == 0, "128-byte swizzle tiles need 1024-byte alignment");
+  static_assert(kSmem <= 227 * 1024, "shared memory budget");
+};
 
 // Scale/bias row of row mblk*128 + r of W_gate (m = 0) or W_up (m = 1) of item wi.
 __device__ __forceinline__ SbRow sb_row_gu(const GemmArgs &a, const WorkItem &wi, int m, int r) {
@@ -97,8 +111,17 @@ __device__ __forceinline__ SbRow sb_row_gu(const GemmArgs &a, const WorkItem &wi
   return SbRow{(sh ? a.w.sh_scales : a.w.scales) + off, (sh ? a.w.sh_biases : a.w.biases) + off, H};
 }
 
-__global__ void __launch_bounds__(kThreads, 1) gemm_gate_up_kernel(const GemmArgs a,
-                                                                   const __grid_constant__ TmaMaps maps) {
+template <int N>
+__global__ void __launch_bounds__(GuTile<N>::kThreads, 1) gemm_gate_up_kernel(const GemmArgs a,
+                                                                              const __grid_constant__ TmaMaps maps) {
+  using C = GuTile<N>;
+  constexpr int kEpiPerQ = C::kEpiPerQ, kDqPerQ = C::kDqPerQ, kEpiWarps = C::kEpiWarps;
+  constexpr int kDqWarp0 = C::kDqWarp0, kDqWarps = C::kDqWarps;
+  constexpr int kN = C::kN, kBStages = C::kBStages, kPkStages = C::kPkStages, kAStages = C::kAStages;
+  constexpr int kBAtomBytes = C::kBAtomBytes, kBStageBytes = C::kBStageBytes, kAccCols = C::kAccCols;
+  constexpr int kACol0 = C::kACol0, kStgBytes = C::kStgBytes;
+  constexpr int kOffPk = C::kOffPk, kOffB = C::kOffB, kOffStg = C::kOffStg, kOffBar = C::kOffBar;
+  constexpr int kOffMisc = C::kOffMisc;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t *sPk = smem + kOffPk;
@@ -282,7 +305,7 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_gate_up_kernel(const GemmArg
     __half *stg = reinterpret_cast<__half *>(smem + kOffStg + q * kStgBytes);
     const int scol = (lane & ~7) + kperm_dst(lane & 7);  // K-permuted order of the down GEMM's operand
     const uint32_t tq = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
-    static_assert(kN == 128, "four 32-token exponent registers per lane");
+    constexpr int kER = kN / 32;  // exponent registers per lane: token 32c + lane in register c
     int li = 0;
     for (int it = blockIdx.x; it < nitems; it += gridDim.x, ++li) {
       const WorkItem wi = a.items[it];
@@ -290,9 +313,9 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_gate_up_kernel(const GemmArg
       const int ng = (wi.nrows + 15) >> 4;  // 16-token groups of the tile
       // exponent of each token's scaling (lane l of register c: token 32c + l),
       // loaded while the accumulators are still being computed
-      int e_l[4];
+      int e_l[kER];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < kER; ++c) {
         const int jl = 32 * c + lane;
         e_l[c] = jl < wi.nrows ? a.row_exp[wi.row0 + jl] : 0;
       }
@@ -318,7 +341,10 @@ __global__ void __launch_bounds__(kThreads, 1) gemm_gate_up_kernel(const GemmArg
           if (lane == 0) mbar_arrive(acc_empty);
         }
         const int ec = g >> 1;
-        const int e_g = ec == 0 ? e_l[0] : ec == 1 ? e_l[1] : ec == 2 ? e_l[2] : e_l[3];
+        int e_g = e_l[0];
+#pragma unroll
+        for (int c = 1; c < kER; ++c)
+          if (ec == c) e_g = e_l[c];
 #pragma unroll
         for (int jj = 0; jj < 16; ++jj) {
           const int e = __shfl_sync(0xffffffffu, e_g, 16 * (g & 1) + jj);
@@ -463,11 +489,18 @@ cudaError_t launch_gemm_gate_up(const GemmArgs &a, int num_sms, cudaStream_t s, 
                       kTileK, CU_TENSOR_MAP_SWIZZLE_128B);
   maps.b_sh = maps.b;
   if (!ok) return cudaErrorInvalidValue;
-  static std::atomic<uint64_t> smem_set{0};
-  const cudaError_t e = ensure_smem_limit(gemm_gate_up_kernel, kSmem, smem_set);
-  if (e != cudaSuccess) return e;
   const int grid = std::max(1, std::min(num_sms, a.max_items));
-  return launch_k(gemm_gate_up_kernel, dim3(grid), dim3(kThreads), kSmem, s, pdl, a, maps);
+  if (a.gu_tile == GuTile<32>::kN) {
+    static std::atomic<uint64_t> smem_set{0};
+    const cudaError_t e = ensure_smem_limit(gemm_gate_up_kernel<32>, GuTile<32>::kSmem, smem_set);
+    if (e != cudaSuccess) return e;
+    return launch_k(gemm_gate_up_kernel<32>, dim3(grid), dim3(GuTile<32>::kThreads), GuTile<32>::kSmem, s, pdl, a, maps);
+  }
+  if (a.gu_tile != GuTile<128>::kN) return cudaErrorInvalidValue;
+  static std::atomic<uint64_t> smem_set{0};
+  const cudaError_t e = ensure_smem_limit(gemm_gate_up_kernel<128>, GuTile<128>::kSmem, smem_set);
+  if (e != cudaSuccess) return e;
+  return launch_k(gemm_gate_up_kernel<128>, dim3(grid), dim3(GuTile<128>::kThreads), GuTile<128>::kSmem, s, pdl, a, maps);
 }
 
 }  // namespace moe

@@ -11,6 +11,13 @@ constexpr int kTileM = 128;   // down GEMM: weight rows per tile (MMA M)
 constexpr int kTileN = 128;   // down GEMM: activation rows per tile (MMA N, max)
 constexpr int kGuTileM = 128; // gate/up GEMM: output rows per tile (the same rows of W_gate and W_up)
 constexpr int kGuTileN = 128; // gate/up GEMM: activation rows per tile (MMA N, max)
+constexpr int kGuTileNSmall = 32;  // the same, when the expert groups are small
+
+// Activation rows per gate/up tile for a batch: the small tile when the
+// groups average at most 32 rows (T*k routed rows over E experts).
+inline int gu_tile_rows(int64_t T, int64_t k, int64_t E) {
+  return T * k <= static_cast<int64_t>(kGuTileNSmall) * E ? kGuTileNSmall : kGuTileN;
+}
 constexpr int kTileK = 64;    // K elements per pipeline stage (one 128-byte fp16 row)
 
 struct RouteScanArgs {
@@ -19,6 +26,7 @@ struct RouteScanArgs {
   int32_t *offsets;     // [E+1]
   WorkItem *gu_items;   // gate/up work list
   int max_gu;
+  int gu_tile;          // activation rows per gate/up tile (down: kTileN)
   WorkItem *dn_items;   // down work list
   int max_dn;
   int32_t *item_counts; // [0] gate/up items, [1] down items
@@ -69,6 +77,7 @@ struct GemmArgs {
   const int32_t *item_count;
   int max_items;
   int64_t xt_rows;          // rows allocated for xt (tensor-map extent)
+  int gu_tile;              // activation rows per gate/up tile (kGuTileN or kGuTileNSmall; down: kTileN)
   int64_t h_rows;           // routed h rows allocated
   int64_t hs_rows;          // shared h rows allocated
   DevStatus *status;

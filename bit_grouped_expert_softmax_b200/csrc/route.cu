@@ -103,7 +103,7 @@ __global__ void __launch_bounds__(256) route_scan_kernel(RouteScanArgs a) {
       int n = 0, gi = 0, di = 0;
       if (g < G) {
         n = (g < E) ? tot[g] : a.T;
-        gi = ((n + kGuTileN - 1) / kGuTileN) * ((g < E ? a.I : a.Is) / kGuTileM);
+        gi = ((n + a.gu_tile - 1) / a.gu_tile) * ((g < E ? a.I : a.Is) / kGuTileM);
         di = ((n + kTileN - 1) / kTileN) * (a.H / kTileM);
       }
       cnt[i] = (g < E) ? n : 0;
@@ -149,12 +149,12 @@ __global__ void __launch_bounds__(256) route_scan_kernel(RouteScanArgs a) {
   for (int g = warp; g < G; g += blockDim.x >> 5) {
     const int n = (g < E) ? tot[g] : a.T;
     const int row0 = (g < E) ? off[g] : R;
-    const int ntg = (n + kGuTileN - 1) / kGuTileN, ntile = (n + kTileN - 1) / kTileN;
+    const int ntg = (n + a.gu_tile - 1) / a.gu_tile, ntile = (n + kTileN - 1) / kTileN;
     const int mg = (g < E ? a.I : a.Is) / kGuTileM, md = a.H / kTileM;
     for (int i = lane; i < ntg * mg; i += 32) {
       const int nt = i / mg, mb = i % mg, slot = gu_off[g] + i;
       if (slot < a.max_gu)
-        a.gu_items[slot] = WorkItem{g, row0 + nt * kGuTileN, min(kGuTileN, n - nt * kGuTileN), mb};
+        a.gu_items[slot] = WorkItem{g, row0 + nt * a.gu_tile, min(a.gu_tile, n - nt * a.gu_tile), mb};
     }
     for (int i = lane; i < ntile * md; i += 32) {
       const int nt = i / md, mb = i % md, slot = dn_off[g] + i;
