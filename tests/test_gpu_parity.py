@@ -195,6 +195,28 @@ def test_forward_host_matches_device_call(name):
         assert np.array_equal(op.view(np.int16), dev), f"pageable call {call}"
 
 
+def test_forward_host_unaligned_pinned_buffers_take_the_copies():
+    """Pinned host buffers that are not 16-byte aligned are not read through
+    the host mapping (the small-batch kernel loads 16 bytes at a time): the
+    call stages them with copies and gives the device call's result."""
+    inp = workload("decode")
+    plan = _plan(inp)
+    layer = _layer(inp)
+    dev = _forward(plan, inp, layer)
+    n = inp.x.size
+    xb = torch.empty(n + 2, dtype=torch.int16).pin_memory()
+    xb[2:] = torch.from_numpy(inp.x.view(np.int16).ravel())
+    lb = torch.empty(inp.logits.size + 1, dtype=torch.float32).pin_memory()
+    lb[1:] = torch.from_numpy(inp.logits.ravel())
+    ob = torch.empty(n + 2, dtype=torch.int16).pin_memory()
+    for call in range(3):
+        ob.fill_(0x7FC0)
+        api.moe_forward_host(plan.handle, inp.T, xb.data_ptr() + 4, lb.data_ptr() + 4, *layer.args(),
+                             ob.data_ptr() + 4)
+        assert np.array_equal(ob[2:].numpy().reshape(dev.shape), dev), f"call {call}"
+    plan.status_sync()
+
+
 def test_output_canaries_untouched():
     inp = workload("tiny")
     plan = _plan(inp)
