@@ -509,27 +509,22 @@ moe_status moe_forward_host(moe_plan_t *plan, int T, const void *x_bf16_host, co
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const size_t xb = static_cast<size_t>(T) * plan->H * 2, lb = static_cast<size_t>(T) * plan->E * 4;
   const LayerWeights w = make_weights(packed_w, scales, biases, shared_packed_w, shared_scales, shared_biases);
-  // the device address of a pinned (page-locked, mapped), 16-byte aligned
-  // host buffer, or null
-  auto mapped = [](const void *ptr) -> void * {
+  // whether a host buffer is pinned (page-locked): copies from it are asynchronous
+  auto mapped = [](const void *ptr) {
     cudaPointerAttributes at;
     if (cudaPointerGetAttributes(&at, ptr) != cudaSuccess) {
       cudaGetLastError();
-      return nullptr;
+      return false;
     }
-    if (at.type != cudaMemoryTypeHost || (reinterpret_cast<uintptr_t>(at.devicePointer) & 15) != 0) return nullptr;
-    return at.devicePointer;
+    return at.type == cudaMemoryTypeHost;
   };
-  void *x_map = mapped(x_bf16_host), *l_map = mapped(router_logits_host), *o_map = mapped(out_bf16_host);
-  // On the small-batch path (a few KB each way) the kernel reads x and the
-  // logits and writes out through the host mapping: no staging copies, the
-  // transfer happens inside the one kernel launch.
-  const bool zero_copy = x_map && l_map && o_map && (use_small_t(plan, T) || (plan->flags & MOE_FLAG_FORCE_SMALL_T));
+  // (the layer's kernels could read the inputs through the host mapping
+  // instead of staged copies, but every CTA of the small-batch kernel reads
+  // all of x and the logits: 148 reads over the host link per call made the
+  // call slower, 65 instead of 45 us at T = 1)
+  const bool pinned_all = mapped(x_bf16_host) && mapped(router_logits_host) && mapped(out_bf16_host);
   // the copies and the layer, enqueued on stream q
   auto enqueue_all = [&](cudaStream_t q) -> moe_status {
-    if (zero_copy)
-      return enqueue_layer(plan, T, static_cast<const uint16_t *>(x_map), static_cast<const float *>(l_map), w,
-                           nullptr, static_cast<uint16_t *>(o_map), q);
     MOE_CUDA(cudaMemcpyAsync(plan->x_stage, x_bf16_host, xb, cudaMemcpyHostToDevice, q), "copy x to device");
     MOE_CUDA(cudaMemcpyAsync(plan->logits_stage, router_logits_host, lb, cudaMemcpyHostToDevice, q),
              "copy logits to device");
@@ -546,7 +541,7 @@ moe_status moe_forward_host(moe_plan_t *plan, int T, const void *x_bf16_host, co
   moe_plan_s::HostKey key = {{x_bf16_host, router_logits_host, out_bf16_host, packed_w, scales, biases,
                               shared_packed_w, shared_scales, shared_biases,
                               reinterpret_cast<const void *>(static_cast<intptr_t>(T))}};
-  const bool graphable = plan->prof_kind.empty() && !plan->test_fault_armed && x_map && l_map && o_map;
+  const bool graphable = plan->prof_kind.empty() && !plan->test_fault_armed && pinned_all;
   if (graphable) {
     for (auto &g : plan->host_graphs)
       if (g.key == key) {

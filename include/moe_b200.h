@@ -193,13 +193,10 @@ moe_status moe_router_logits(moe_plan_t *plan, int T, const void *x_bf16, const 
  * out_bf16_host are host pointers (pinned memory gives asynchronous copies);
  * the weights are device pointers. Copies the inputs into the plan's device
  * staging buffers, runs the layer, copies the output back and waits for the
- * stream, so the host buffers may be reused on return. When the batch takes
- * the small-batch kernel (T <= 8) and all three host buffers are pinned
- * (page-locked and mapped, e.g. cudaHostAlloc) and 16-byte aligned, there
- * are no staging copies: the kernel reads x and the logits and writes the
- * output through the host mapping. With pinned host buffers, a call whose
- * arguments (buffers, weights, T) the plan has seen before is captured into
- * a CUDA graph and replayed on later such calls (one launch), for up to 64
+ * stream, so the host buffers may be reused on return. With pinned host
+ * buffers, a call whose arguments (buffers, weights, T) the plan has seen
+ * before is captured into a CUDA graph and replayed on later such calls (one
+ * launch instead of three copies and the layer's kernels), for up to 64
  * argument sets (a decode loop over a model's layers); results are the same.
  * Not while profiling is enabled.
  */

@@ -195,10 +195,10 @@ def test_forward_host_matches_device_call(name):
         assert np.array_equal(op.view(np.int16), dev), f"pageable call {call}"
 
 
-def test_forward_host_unaligned_pinned_buffers_take_the_copies():
-    """Pinned host buffers that are not 16-byte aligned are not read through
-    the host mapping (the small-batch kernel loads 16 bytes at a time): the
-    call stages them with copies and gives the device call's result."""
+def test_forward_host_unaligned_pinned_buffers():
+    """Pinned host buffers at addresses that are not 16-byte aligned: the
+    call stages them into aligned device buffers and gives the device call's
+    result, eagerly and from its captured graph."""
     inp = workload("decode")
     plan = _plan(inp)
     layer = _layer(inp)
