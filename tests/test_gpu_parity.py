@@ -108,6 +108,15 @@ def test_forward_mid_size_ragged():
     check_output(_forward(_plan(inp), inp), oracle.moe_forward(inp), "mid")
 
 
+@pytest.mark.parametrize("T", [256, 257])
+def test_gate_up_tile_choice_boundary(T):
+    """The gate/up GEMM takes 32-row tiles while the groups average at most 32
+    rows (T*k <= 32*E) and 128-row tiles above: both sides of the boundary,
+    with ragged groups of both sizes."""
+    inp = synth.make_layer(T, 512, 32, 4, 256, 384, seed=40 + T, logit_std=1.5)
+    check_output(_forward(_plan(inp), inp), oracle.moe_forward(inp), f"T={T}")
+
+
 @pytest.mark.parametrize("name", ["prefill", "zipf"])
 def test_forward_full_size_every_row(name):
     """Every token row of the full-size layer against the oracle (the by-expert
