@@ -509,22 +509,38 @@ moe_status moe_forward_host(moe_plan_t *plan, int T, const void *x_bf16_host, co
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const size_t xb = static_cast<size_t>(T) * plan->H * 2, lb = static_cast<size_t>(T) * plan->E * 4;
   const LayerWeights w = make_weights(packed_w, scales, biases, shared_packed_w, shared_scales, shared_biases);
-  // whether a host buffer is pinned (page-locked): copies from it are asynchronous
-  auto mapped = [](const void *ptr) {
+  // the device address of a pinned (page-locked, mapped) host buffer aligned
+  // to `align` bytes, or null
+  auto mapped = [](const void *ptr, uintptr_t align) -> void * {
     cudaPointerAttributes at;
     if (cudaPointerGetAttributes(&at, ptr) != cudaSuccess) {
       cudaGetLastError();
-      return false;
+      return nullptr;
     }
-    return at.type == cudaMemoryTypeHost;
+    if (at.type != cudaMemoryTypeHost || !at.devicePointer) return nullptr;
+    return (reinterpret_cast<uintptr_t>(at.devicePointer) % align) == 0 ? at.devicePointer : nullptr;
   };
-  // (the layer's kernels could read the inputs through the host mapping
-  // instead of staged copies, but every CTA of the small-batch kernel reads
-  // all of x and the logits: 148 reads over the host link per call made the
-  // call slower, 65 instead of 45 us at T = 1)
-  const bool pinned_all = mapped(x_bf16_host) && mapped(router_logits_host) && mapped(out_bf16_host);
+  void *x_map = mapped(x_bf16_host, 16), *l_map = mapped(router_logits_host, 4), *o_map = mapped(out_bf16_host, 16);
+  const bool pinned_all = x_map && l_map && o_map;
+  // On the small-batch path one block reads the inputs through the host
+  // mapping into the staging buffers and the kernel writes its output straight
+  // into the host buffer: two short kernels instead of three copies and the
+  // kernel. (Letting the kernel read x and the logits through the mapping
+  // itself was slower: every one of its CTAs reads all of them.)
+  const bool host_direct = pinned_all && (use_small_t(plan, T) || (plan->flags & MOE_FLAG_FORCE_SMALL_T));
   // the copies and the layer, enqueued on stream q
   auto enqueue_all = [&](cudaStream_t q) -> moe_status {
+    if (host_direct) {
+      HostStageArgs hs{};
+      hs.x_host = static_cast<const uint4 *>(x_map);
+      hs.x_dev = reinterpret_cast<uint4 *>(plan->x_stage);
+      hs.x16 = static_cast<int>(xb / 16);
+      hs.l_host = static_cast<const uint32_t *>(l_map);
+      hs.l_dev = reinterpret_cast<uint32_t *>(plan->logits_stage);
+      hs.l4 = static_cast<int>(lb / 4);
+      MOE_CUDA(launch_host_stage(hs, q, pdl(plan)), "host staging launch");
+      return enqueue_layer(plan, T, plan->x_stage, plan->logits_stage, w, nullptr, static_cast<uint16_t *>(o_map), q);
+    }
     MOE_CUDA(cudaMemcpyAsync(plan->x_stage, x_bf16_host, xb, cudaMemcpyHostToDevice, q), "copy x to device");
     MOE_CUDA(cudaMemcpyAsync(plan->logits_stage, router_logits_host, lb, cudaMemcpyHostToDevice, q),
              "copy logits to device");

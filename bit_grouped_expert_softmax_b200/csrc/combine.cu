@@ -61,6 +61,20 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
   }
 }
 
+// One block copies a host-buffer call's inputs (pinned host memory, read
+// through the host mapping once) into the plan's device staging buffers;
+// n16: 16-byte chunks, tail: the last bytes of the logits, 4 at a time.
+__global__ void __launch_bounds__(256) host_stage_kernel(HostStageArgs a) {
+  pdl_wait();  // the staging buffers may still be read by the kernel ahead
+  pdl_trigger();
+  for (int i = threadIdx.x; i < a.x16; i += blockDim.x) a.x_dev[i] = a.x_host[i];
+  for (int i = threadIdx.x; i < a.l4; i += blockDim.x) a.l_dev[i] = a.l_host[i];
+}
+
+cudaError_t launch_host_stage(const HostStageArgs &a, cudaStream_t s, bool pdl) {
+  return launch_k(host_stage_kernel, dim3(1), dim3(256), 0, s, pdl, a);
+}
+
 cudaError_t launch_combine(const CombineArgs &a, cudaStream_t s, bool pdl) {
   if (a.T <= 0) return cudaSuccess;
   return launch_k(combine_kernel, dim3(a.T), dim3(256), 0, s, pdl, a);

@@ -117,6 +117,17 @@ struct SmallTArgs {
   int test_fault;           // testing only: row block 0 of the shared expert does not publish its h
 };
 
+// A host-buffer call's inputs, from their host mapping to the device staging
+// buffers (x in 16-byte chunks, the logits in 4-byte words).
+struct HostStageArgs {
+  const uint4 *x_host;
+  uint4 *x_dev;
+  int x16;
+  const uint32_t *l_host;
+  uint32_t *l_dev;
+  int l4;
+};
+
 struct RouterArgs {
   int T, E, H;
   const uint16_t *x;        // [T, H] bf16
@@ -155,6 +166,7 @@ cudaError_t launch_gemm_gate_up(const GemmArgs &a, int num_sms, cudaStream_t s, 
 cudaError_t launch_gemm_down(const GemmArgs &a, int num_sms, cudaStream_t s, bool pdl);
 cudaError_t launch_combine(const CombineArgs &a, cudaStream_t s, bool pdl);
 cudaError_t launch_router(const RouterArgs &a, cudaStream_t s, bool pdl);
+cudaError_t launch_host_stage(const HostStageArgs &a, cudaStream_t s, bool pdl);
 cudaError_t launch_small_t(const SmallTArgs &a, int num_sms, cudaStream_t s, bool pdl);
 int small_t_grid(int num_sms);
 // whether the fused small-T kernel can run this layer (shared memory, grid)

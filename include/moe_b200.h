@@ -193,11 +193,16 @@ moe_status moe_router_logits(moe_plan_t *plan, int T, const void *x_bf16, const 
  * out_bf16_host are host pointers (pinned memory gives asynchronous copies);
  * the weights are device pointers. Copies the inputs into the plan's device
  * staging buffers, runs the layer, copies the output back and waits for the
- * stream, so the host buffers may be reused on return. With pinned host
- * buffers, a call whose arguments (buffers, weights, T) the plan has seen
- * before is captured into a CUDA graph and replayed on later such calls (one
- * launch instead of three copies and the layer's kernels), for up to 64
- * argument sets (a decode loop over a model's layers); results are the same.
+ * stream, so the host buffers may be reused on return. When the batch takes
+ * the small-batch kernel (T <= 8) and the three host buffers are pinned
+ * (page-locked and mapped, e.g. cudaHostAlloc), with x and out 16-byte and
+ * the logits 4-byte aligned, one block reads the inputs through the host
+ * mapping into the staging buffers and the kernel writes the output straight
+ * into out_bf16_host (no copy engine involved). With pinned host buffers, a
+ * call whose arguments (buffers, weights, T) the plan has seen before is
+ * captured into a CUDA graph and replayed on later such calls (one launch),
+ * for up to 64 argument sets (a decode loop over a model's layers); results
+ * are the same.
  * Not while profiling is enabled.
  */
 moe_status moe_forward_host(moe_plan_t *plan, int T, const void *x_bf16_host,
