@@ -146,20 +146,42 @@ __global__ void __launch_bounds__(256) route_scan_kernel(RouteScanArgs a) {
     a.item_counts[1] = min(dn_total, a.max_dn);
     *a.done = 0;  // ready for the next launch (the kernel boundary orders it)
   }
+  // (n-tile, m-block) of item i is (i / m, i % m); lane l starts at item l
+  // and steps by 32 items, so the quotient and remainder are carried along
+  // instead of divided out per item
   for (int g = warp; g < G; g += blockDim.x >> 5) {
     const int n = (g < E) ? tot[g] : a.T;
     const int row0 = (g < E) ? off[g] : R;
     const int ntg = (n + a.gu_tile - 1) / a.gu_tile, ntile = (n + kTileN - 1) / kTileN;
     const int mg = (g < E ? a.I : a.Is) / kGuTileM, md = a.H / kTileM;
-    for (int i = lane; i < ntg * mg; i += 32) {
-      const int nt = i / mg, mb = i % mg, slot = gu_off[g] + i;
-      if (slot < a.max_gu)
-        a.gu_items[slot] = WorkItem{g, row0 + nt * a.gu_tile, min(a.gu_tile, n - nt * a.gu_tile), mb};
+    {
+      int nt = lane / mg, mb = lane % mg;
+      const int qs = 32 / mg, rs = 32 % mg;
+      for (int i = lane; i < ntg * mg; i += 32) {
+        const int slot = gu_off[g] + i;
+        if (slot < a.max_gu)
+          a.gu_items[slot] = WorkItem{g, row0 + nt * a.gu_tile, min(a.gu_tile, n - nt * a.gu_tile), mb};
+        nt += qs;
+        mb += rs;
+        if (mb >= mg) {
+          mb -= mg;
+          ++nt;
+        }
+      }
     }
-    for (int i = lane; i < ntile * md; i += 32) {
-      const int nt = i / md, mb = i % md, slot = dn_off[g] + i;
-      if (slot < a.max_dn)
-        a.dn_items[slot] = WorkItem{g, row0 + nt * kTileN, min(kTileN, n - nt * kTileN), mb};
+    {
+      int nt = lane / md, mb = lane % md;
+      const int qs = 32 / md, rs = 32 % md;
+      for (int i = lane; i < ntile * md; i += 32) {
+        const int slot = dn_off[g] + i;
+        if (slot < a.max_dn) a.dn_items[slot] = WorkItem{g, row0 + nt * kTileN, min(kTileN, n - nt * kTileN), mb};
+        nt += qs;
+        mb += rs;
+        if (mb >= md) {
+          mb -= md;
+          ++nt;
+        }
+      }
     }
   }
 }
@@ -168,17 +190,20 @@ __global__ void __launch_bounds__(256) route_scan_kernel(RouteScanArgs a) {
 // bases is reset to zero afterwards, ready for the next routing's histogram.
 __global__ void __launch_bounds__(256) route_scatter_kernel(RouteScatterArgs a) {
   __shared__ int cnt[kMaxExperts];
+  __shared__ int sid[kRouteChunk * kMaxTopK];  // the chunk's expert ids, flat order
   pdl_wait();
   pdl_trigger();
   const int chunk = blockIdx.x, E = a.E, k = a.k, T = a.T;
   int32_t *row = a.chunk_base + static_cast<size_t>(chunk) * E;
-  // the chunk's first row of each expert: the expert's offset plus the
-  // entries of earlier chunks (the scan's per-chunk prefix)
-  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = __ldcg(row + e) + __ldcg(a.offsets + e);
-  __syncthreads();
-  for (int e = threadIdx.x; e < E; e += blockDim.x) row[e] = 0;
   const int t0 = chunk * kRouteChunk, t1 = min(T, t0 + kRouteChunk);
   const int f0 = t0 * k, f1 = t1 * k;
+  // the chunk's first row of each expert: the expert's offset plus the
+  // entries of earlier chunks (the scan's per-chunk prefix); and the chunk's
+  // ids, all loaded by the whole block at once
+  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = __ldcg(row + e) + __ldcg(a.offsets + e);
+  for (int f = f0 + threadIdx.x; f < f1; f += blockDim.x) sid[f - f0] = a.ids[f];
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) row[e] = 0;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (warp != 0) return;
   // flat order f = t*k + j is token-ascending; within a batch of 32 entries the
@@ -188,7 +213,7 @@ __global__ void __launch_bounds__(256) route_scatter_kernel(RouteScatterArgs a) 
     const bool valid = f < f1;
     const unsigned active = __ballot_sync(0xffffffffu, valid);
     if (valid) {
-      const int e = a.ids[f];
+      const int e = sid[f - f0];
       const unsigned peers = __match_any_sync(active, e);
       const int rank = __popc(peers & ((1u << lane) - 1u));
       const int base = cnt[e];
