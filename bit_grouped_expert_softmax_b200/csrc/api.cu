@@ -93,7 +93,7 @@ struct moe_plan_s {
   WorkItem *gu_items;
   WorkItem *dn_items;
   int32_t *item_counts;
-  int32_t *scan_done;
+  int32_t *totals;
   __half *xt;
   __half *h;
   __half *y;
@@ -206,19 +206,18 @@ moe_status enqueue_routing(moe_plan_s *p, int T, const float *logits, const uint
              "route_topk launch");
   }
   RouteScanArgs sa{};
-  sa.T = T; sa.E = p->E; sa.k = p->k; sa.H = p->H; sa.I = p->I; sa.Is = p->Is; sa.nchunk = nchunk;
-  sa.chunk_cnt = p->chunk; sa.offsets = p->offsets;
-  sa.gu_items = p->gu_items; sa.max_gu = static_cast<int>(p->max_gu); sa.gu_tile = gu_tile_rows(T, p->k, p->E);
-  sa.dn_items = p->dn_items; sa.max_dn = static_cast<int>(p->max_dn);
-  sa.item_counts = p->item_counts; sa.done = p->scan_done; sa.status = p->status;
+  sa.E = p->E; sa.nchunk = nchunk; sa.chunk_cnt = p->chunk; sa.totals = p->totals;
   {
     ProfScope ps(p, MOE_KERNEL_ROUTE_SCAN, s);
     MOE_CUDA(launch_k(route_scan_kernel, dim3(static_cast<int>(cdiv(p->E, 8))), dim3(256), 0, s, pdl(p), sa),
              "route_scan launch");
   }
   RouteScatterArgs ca{};
-  ca.T = T; ca.E = p->E; ca.k = p->k; ca.H = p->H;
-  ca.ids = p->ids; ca.chunk_base = p->chunk; ca.offsets = p->offsets; ca.perm = p->perm; ca.inv = p->inv;
+  ca.T = T; ca.E = p->E; ca.k = p->k; ca.H = p->H; ca.I = p->I; ca.Is = p->Is;
+  ca.ids = p->ids; ca.chunk_base = p->chunk; ca.totals = p->totals; ca.offsets = p->offsets; ca.perm = p->perm;
+  ca.inv = p->inv;
+  ca.gu_items = p->gu_items; ca.max_gu = static_cast<int>(p->max_gu); ca.gu_tile = gu_tile_rows(T, p->k, p->E);
+  ca.dn_items = p->dn_items; ca.max_dn = static_cast<int>(p->max_dn); ca.item_counts = p->item_counts;
   ca.x = x; ca.xt = p->xt; ca.xexp = p->xexp; ca.status = p->status;
   ca.wts = p->wts; ca.row_exp = p->row_exp; ca.row_w = p->row_w;
   {
@@ -364,7 +363,7 @@ moe_status moe_plan(int T_max, int hidden, int n_experts, int top_k, int inter, 
       static_cast<size_t>(p->max_gu) * sizeof(WorkItem),
       static_cast<size_t>(p->max_dn) * sizeof(WorkItem),
       16,                                    // item counts
-      16,                                    // scan: blocks finished
+      E * 4,                                 // rows routed to each expert
       (R + T) * H * 2,                       // xt
       (R * I + T * Is) * 2,                  // h
       (R + T) * H * 2,                       // y
@@ -402,7 +401,7 @@ moe_status moe_plan(int T_max, int hidden, int n_experts, int top_k, int inter, 
   p->gu_items = reinterpret_cast<WorkItem *>(b + offs[i++]);
   p->dn_items = reinterpret_cast<WorkItem *>(b + offs[i++]);
   p->item_counts = reinterpret_cast<int32_t *>(b + offs[i++]);
-  p->scan_done = reinterpret_cast<int32_t *>(b + offs[i++]);
+  p->totals = reinterpret_cast<int32_t *>(b + offs[i++]);
   p->xt = reinterpret_cast<__half *>(b + offs[i++]);
   p->h = reinterpret_cast<__half *>(b + offs[i++]);
   p->y = reinterpret_cast<__half *>(b + offs[i++]);

@@ -21,24 +21,23 @@ inline int gu_tile_rows(int64_t T, int64_t k, int64_t E) {
 constexpr int kTileK = 64;    // K elements per pipeline stage (one 128-byte fp16 row)
 
 struct RouteScanArgs {
-  int T, E, k, H, I, Is, nchunk;
-  int32_t *chunk_cnt;   // [nchunk][E] counts in, bases out
-  int32_t *offsets;     // [E+1]
-  WorkItem *gu_items;   // gate/up work list
-  int max_gu;
-  int gu_tile;          // activation rows per gate/up tile (down: kTileN)
-  WorkItem *dn_items;   // down work list
-  int max_dn;
-  int32_t *item_counts; // [0] gate/up items, [1] down items
-  int32_t *done;        // blocks finished (zero between launches)
-  DevStatus *status;
+  int E, nchunk;
+  int32_t *chunk_cnt;   // [nchunk][E] counts in, per-chunk prefixes out
+  int32_t *totals;      // [E] rows routed to each expert
 };
 
 struct RouteScatterArgs {
-  int T, E, k, H;
+  int T, E, k, H, I, Is;
   const int32_t *ids;         // [T*k]
   int32_t *chunk_base;        // [nchunk][E] per-chunk prefixes in; zeroed on the way out
-  const int32_t *offsets;     // [E+1] first row of each expert
+  const int32_t *totals;      // [E] rows routed to each expert
+  int32_t *offsets;           // [E+1] first row of each expert (written by block 0)
+  WorkItem *gu_items;         // gate/up work list
+  int max_gu;
+  int gu_tile;                // activation rows per gate/up tile (down: kTileN)
+  WorkItem *dn_items;         // down work list
+  int max_dn;
+  int32_t *item_counts;       // [0] gate/up items, [1] down items (written by block 0)
   int32_t *perm;              // [T*k]
   int32_t *inv;               // [T*k]
   const uint16_t *x;          // [T, H] bf16, or null (routing only)

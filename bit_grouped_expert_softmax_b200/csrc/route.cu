@@ -8,11 +8,13 @@
 //   route_topk_kernel    softmax over E, warp top-k, renormalised weights,
 //                        per-chunk expert histogram
 //   route_scan_kernel    per-expert totals and per-chunk prefixes (one warp per
-//                        expert), then, in the last block to finish, the
-//                        exclusive scan (offsets) and the grouped-GEMM work
-//                        lists (block map)
-//   route_scatter_kernel stable permutation (experts ascending, tokens ascending
-//                        within an expert) and its inverse
+//                        expert)
+//   route_scatter_kernel the exclusive scan of the totals (offsets) and the
+//                        grouped-GEMM work lists (block map), each block
+//                        computing the scan itself and writing its share of
+//                        the lists; the stable permutation (experts
+//                        ascending, tokens ascending within an expert) and its
+//                        inverse
 //   gather_kernel        each token's row, fp16 scaled by a power of two, copied
 //                        to its k routed rows and its shared-expert row (expert-
 //                        contiguous, the gate/up GEMM's activation operand), and
@@ -47,69 +49,82 @@ __global__ void __launch_bounds__(256) route_topk_kernel(int T, int E, int k,
 // One warp per expert (8 per block). Each warp turns its expert's column of
 // per-chunk counts into exclusive prefix sums over the chunks (in place: the
 // rows each chunk's first entry lands at, relative to the expert's first row)
-// and leaves the expert's total in offsets[e]. The last block to finish
-// (counted in *done) scans the totals into offsets[0..E] and writes the two
-// work lists (block map), then resets *done for the next launch.
+// and leaves the expert's total in totals[e].
 __global__ void __launch_bounds__(256) route_scan_kernel(RouteScanArgs a) {
-  __shared__ int off[kMaxExperts + 2];
-  __shared__ int gu_off[kMaxExperts + 2];
-  __shared__ int dn_off[kMaxExperts + 2];
-  __shared__ int tot[kMaxExperts + 1];
-  __shared__ int totals3[3];
-  __shared__ int is_last;
   pdl_wait();
   pdl_trigger();
   const int E = a.E;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int e = blockIdx.x * 8 + warp;
-  if (e < E) {
-    int run = 0;
-    for (int c0 = 0; c0 < a.nchunk; c0 += 128) {
-      int v[4];
+  if (e >= E) return;
+  int run = 0;
+  for (int c0 = 0; c0 < a.nchunk; c0 += 128) {
+    int v[4];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {  // four loads in flight per lane
-        const int c = c0 + 32 * u + lane;
-        v[u] = c < a.nchunk ? __ldcg(a.chunk_cnt + static_cast<size_t>(c) * E + e) : 0;
-      }
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int c = c0 + 32 * u + lane;
-        const int incl = warp_incl_scan(v[u]);
-        if (c < a.nchunk) a.chunk_cnt[static_cast<size_t>(c) * E + e] = run + incl - v[u];
-        run += __shfl_sync(0xffffffffu, incl, 31);
-      }
+    for (int u = 0; u < 4; ++u) {  // four loads in flight per lane
+      const int c = c0 + 32 * u + lane;
+      v[u] = c < a.nchunk ? __ldcg(a.chunk_cnt + static_cast<size_t>(c) * E + e) : 0;
     }
-    if (lane == 0) a.offsets[e] = run;  // the expert's total until the last block scans them
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int c = c0 + 32 * u + lane;
+      const int incl = warp_incl_scan(v[u]);
+      if (c < a.nchunk) a.chunk_cnt[static_cast<size_t>(c) * E + e] = run + incl - v[u];
+      run += __shfl_sync(0xffffffffu, incl, 31);
+    }
   }
-  __threadfence();  // this thread's prefixes and total are visible before the block counts itself done
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    is_last = atomicAdd(a.done, 1) == static_cast<int>(gridDim.x) - 1;
-  }
-  __syncthreads();
-  if (!is_last) return;
-  __threadfence();
-  for (int g = threadIdx.x; g < E; g += blockDim.x) tot[g] = __ldcg(a.offsets + g);
-  __syncthreads();
+  if (lane == 0) a.totals[e] = run;
+}
+
+// Stable scatter and the block map. One block per routing chunk of 32 tokens.
+// Every block scans the experts' totals into their first rows (offsets) and
+// the groups' work-item counts into list positions itself (257 values, in
+// shared memory: no block waits for another); block 0 stores the offsets and
+// the item counts, and each block writes the work items of every
+// gridDim.x-th group. Warp 0 then ranks the chunk's entries; the chunk's row
+// of bases is reset to zero afterwards, ready for the next routing's
+// histogram. Work items of group g are (n-tile, m-block) with the m-block
+// fastest, so neighbouring CTAs share the activation tile of one n-tile.
+__global__ void __launch_bounds__(256) route_scatter_kernel(RouteScatterArgs a) {
+  __shared__ int cnt[kMaxExperts];
+  __shared__ int sid[kRouteChunk * kMaxTopK];  // the chunk's expert ids, flat order
+  __shared__ int tot[kMaxExperts + 1];
+  __shared__ int off[kMaxExperts + 2], gu_off[kMaxExperts + 2], dn_off[kMaxExperts + 2];
+  __shared__ int totals3[3];
+  pdl_wait();
+  pdl_trigger();
+  const int chunk = blockIdx.x, E = a.E, k = a.k, T = a.T;
   const int G = E + 1;  // routed experts plus the shared one
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int32_t *row = a.chunk_base + static_cast<size_t>(chunk) * E;
+  const int t0 = chunk * kRouteChunk, t1 = min(T, t0 + kRouteChunk);
+  const int f0 = t0 * k, f1 = t1 * k;
+  // the experts' totals, the chunk's per-expert prefix and the chunk's ids,
+  // all loaded by the whole block at once
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    tot[e] = __ldcg(a.totals + e);
+    cnt[e] = __ldcg(row + e);
+  }
+  for (int f = f0 + threadIdx.x; f < f1; f += blockDim.x) sid[f - f0] = a.ids[f];
+  __syncthreads();
   // exclusive scans over the groups, done by warp 0 with 9 values per lane (G <= 257)
   if (warp == 0) {
     constexpr int PER = (kMaxExperts + 1 + 31) / 32;
-    int cnt[PER], gu[PER], dn[PER];
+    int c3[PER], gu[PER], dn[PER];
     int sc = 0, sg = 0, sd = 0;
 #pragma unroll
     for (int i = 0; i < PER; ++i) {
       const int g = lane * PER + i;
       int n = 0, gi = 0, di = 0;
       if (g < G) {
-        n = (g < E) ? tot[g] : a.T;
+        n = (g < E) ? tot[g] : T;
         gi = ((n + a.gu_tile - 1) / a.gu_tile) * ((g < E ? a.I : a.Is) / kGuTileM);
         di = ((n + kTileN - 1) / kTileN) * (a.H / kTileM);
       }
-      cnt[i] = (g < E) ? n : 0;
+      c3[i] = (g < E) ? n : 0;
       gu[i] = gi;
       dn[i] = di;
-      sc += cnt[i];
+      sc += c3[i];
       sg += gi;
       sd += di;
     }
@@ -123,7 +138,7 @@ __global__ void __launch_bounds__(256) route_scan_kernel(RouteScanArgs a) {
         gu_off[g] = bg;
         dn_off[g] = bd;
       }
-      bc += cnt[i];
+      bc += c3[i];
       bg += gu[i];
       bd += dn[i];
     }
@@ -134,78 +149,65 @@ __global__ void __launch_bounds__(256) route_scan_kernel(RouteScanArgs a) {
     }
   }
   __syncthreads();
-  for (int g = threadIdx.x; g <= E; g += blockDim.x) a.offsets[g] = (g < E) ? off[g] : a.T * a.k;
-  // work lists: group g's tiles are (n-tile, m-block) with the m-block fastest,
-  // so neighbouring CTAs share the activation tile of one n-tile
-  const int R = a.T * a.k;
-  const int gu_total = totals3[1], dn_total = totals3[2];
-  if (threadIdx.x == 0) {
-    if (gu_total > a.max_gu || dn_total > a.max_dn)
-      report_error(a.status, kDevBounds, 10, static_cast<uint32_t>(max(gu_total, dn_total)));
-    a.item_counts[0] = min(gu_total, a.max_gu);
-    a.item_counts[1] = min(dn_total, a.max_dn);
-    *a.done = 0;  // ready for the next launch (the kernel boundary orders it)
-  }
-  // (n-tile, m-block) of item i is (i / m, i % m); lane l starts at item l
-  // and steps by 32 items, so the quotient and remainder are carried along
-  // instead of divided out per item
-  for (int g = warp; g < G; g += blockDim.x >> 5) {
-    const int n = (g < E) ? tot[g] : a.T;
-    const int row0 = (g < E) ? off[g] : R;
-    const int ntg = (n + a.gu_tile - 1) / a.gu_tile, ntile = (n + kTileN - 1) / kTileN;
-    const int mg = (g < E ? a.I : a.Is) / kGuTileM, md = a.H / kTileM;
-    {
-      int nt = lane / mg, mb = lane % mg;
-      const int qs = 32 / mg, rs = 32 % mg;
-      for (int i = lane; i < ntg * mg; i += 32) {
-        const int slot = gu_off[g] + i;
-        if (slot < a.max_gu)
-          a.gu_items[slot] = WorkItem{g, row0 + nt * a.gu_tile, min(a.gu_tile, n - nt * a.gu_tile), mb};
-        nt += qs;
-        mb += rs;
-        if (mb >= mg) {
-          mb -= mg;
-          ++nt;
-        }
-      }
-    }
-    {
-      int nt = lane / md, mb = lane % md;
-      const int qs = 32 / md, rs = 32 % md;
-      for (int i = lane; i < ntile * md; i += 32) {
-        const int slot = dn_off[g] + i;
-        if (slot < a.max_dn) a.dn_items[slot] = WorkItem{g, row0 + nt * kTileN, min(kTileN, n - nt * kTileN), mb};
-        nt += qs;
-        mb += rs;
-        if (mb >= md) {
-          mb -= md;
-          ++nt;
-        }
-      }
-    }
-  }
-}
-
-// Stable scatter. One block per routing chunk of 32 tokens. The chunk's row of
-// bases is reset to zero afterwards, ready for the next routing's histogram.
-__global__ void __launch_bounds__(256) route_scatter_kernel(RouteScatterArgs a) {
-  __shared__ int cnt[kMaxExperts];
-  __shared__ int sid[kRouteChunk * kMaxTopK];  // the chunk's expert ids, flat order
-  pdl_wait();
-  pdl_trigger();
-  const int chunk = blockIdx.x, E = a.E, k = a.k, T = a.T;
-  int32_t *row = a.chunk_base + static_cast<size_t>(chunk) * E;
-  const int t0 = chunk * kRouteChunk, t1 = min(T, t0 + kRouteChunk);
-  const int f0 = t0 * k, f1 = t1 * k;
   // the chunk's first row of each expert: the expert's offset plus the
-  // entries of earlier chunks (the scan's per-chunk prefix); and the chunk's
-  // ids, all loaded by the whole block at once
-  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = __ldcg(row + e) + __ldcg(a.offsets + e);
-  for (int f = f0 + threadIdx.x; f < f1; f += blockDim.x) sid[f - f0] = a.ids[f];
+  // entries of earlier chunks (the scan's per-chunk prefix)
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    cnt[e] += off[e];
+    row[e] = 0;
+  }
+  const int R = T * k;
+  if (blockIdx.x == 0) {
+    for (int g = threadIdx.x; g <= E; g += blockDim.x) a.offsets[g] = (g < E) ? off[g] : R;
+    if (threadIdx.x == 0) {
+      const int gu_total = totals3[1], dn_total = totals3[2];
+      if (gu_total > a.max_gu || dn_total > a.max_dn)
+        report_error(a.status, kDevBounds, 10, static_cast<uint32_t>(max(gu_total, dn_total)));
+      a.item_counts[0] = min(gu_total, a.max_gu);
+      a.item_counts[1] = min(dn_total, a.max_dn);
+    }
+  }
   __syncthreads();
-  for (int e = threadIdx.x; e < E; e += blockDim.x) row[e] = 0;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (warp != 0) return;
+  if (warp != 0) {
+    // work items: warps 1..7 of block b take groups b + gridDim.x * j. The
+    // (n-tile, m-block) of item i is (i / m, i % m); lane l starts at item l
+    // and steps by 32 items, carrying quotient and remainder along.
+    for (int g = blockIdx.x + gridDim.x * (warp - 1); g < G; g += gridDim.x * ((blockDim.x >> 5) - 1)) {
+      const int n = (g < E) ? tot[g] : T;
+      const int row0 = (g < E) ? off[g] : R;
+      const int ntg = (n + a.gu_tile - 1) / a.gu_tile, ntile = (n + kTileN - 1) / kTileN;
+      const int mg = (g < E ? a.I : a.Is) / kGuTileM, md = a.H / kTileM;
+      {
+        int nt = lane / mg, mb = lane % mg;
+        const int qs = 32 / mg, rs = 32 % mg;
+        for (int i = lane; i < ntg * mg; i += 32) {
+          const int slot = gu_off[g] + i;
+          if (slot < a.max_gu)
+            a.gu_items[slot] = WorkItem{g, row0 + nt * a.gu_tile, min(a.gu_tile, n - nt * a.gu_tile), mb};
+          nt += qs;
+          mb += rs;
+          if (mb >= mg) {
+            mb -= mg;
+            ++nt;
+          }
+        }
+      }
+      {
+        int nt = lane / md, mb = lane % md;
+        const int qs = 32 / md, rs = 32 % md;
+        for (int i = lane; i < ntile * md; i += 32) {
+          const int slot = dn_off[g] + i;
+          if (slot < a.max_dn) a.dn_items[slot] = WorkItem{g, row0 + nt * kTileN, min(kTileN, n - nt * kTileN), mb};
+          nt += qs;
+          mb += rs;
+          if (mb >= md) {
+            mb -= md;
+            ++nt;
+          }
+        }
+      }
+    }
+    return;
+  }
   // flat order f = t*k + j is token-ascending; within a batch of 32 entries the
   // rank among equal experts comes from match/popc, across batches from cnt[]
   for (int fb = f0; fb < f1; fb += 32) {
