@@ -198,10 +198,11 @@ struct ProfScope {
 // routing kernels: ids/weights + histogram, scan + work lists, scatter, gather (if x)
 moe_status enqueue_routing(moe_plan_s *p, int T, const float *logits, const uint16_t *x, cudaStream_t s) {
   const int nchunk = static_cast<int>(cdiv(T, kRouteChunk));
-  const int tok_blocks = static_cast<int>(cdiv(T, 8));
+  // one warp per token, two per block: a few hundred tokens still spread over every SM
+  const int tok_blocks = static_cast<int>(cdiv(T, 2));
   {
     ProfScope ps(p, MOE_KERNEL_ROUTE_TOPK, s);
-    MOE_CUDA(launch_k(route_topk_kernel, dim3(tok_blocks), dim3(256), 0, s, pdl(p), T, p->E, p->k, logits, p->ids,
+    MOE_CUDA(launch_k(route_topk_kernel, dim3(tok_blocks), dim3(64), 0, s, pdl(p), T, p->E, p->k, logits, p->ids,
                       p->wts, p->chunk),
              "route_topk launch");
   }
@@ -226,7 +227,7 @@ moe_status enqueue_routing(moe_plan_s *p, int T, const float *logits, const uint
   }
   if (x) {
     ProfScope ps(p, MOE_KERNEL_GATHER, s);
-    MOE_CUDA(launch_k(gather_kernel, dim3(tok_blocks), dim3(256), 0, s, pdl(p), ca), "gather launch");
+    MOE_CUDA(launch_k(gather_kernel, dim3(tok_blocks), dim3(64), 0, s, pdl(p), ca), "gather launch");
   }
   return MOE_OK;
 }
