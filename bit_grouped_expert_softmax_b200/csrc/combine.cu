@@ -10,6 +10,11 @@
 
 namespace moe {
 
+// U rows of a chunk are requested before any of them is added (the adds stay
+// in slot order): U = 1 streams one row at a time, which suits the DRAM when
+// thousands of tokens keep it busy; a few hundred tokens leave each SM a
+// handful of blocks, whose row-by-row round trips then set the time.
+template <int U>
 __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
   pdl_wait();
   pdl_trigger();
@@ -31,15 +36,26 @@ __global__ void __launch_bounds__(256) combine_kernel(CombineArgs a) {
     float acc[8];
 #pragma unroll
     for (int q = 0; q < 8; ++q) acc[q] = 0.f;
-    for (int j = 0; j <= k; ++j) {
-      if (rows[j] < 0) continue;
-      const uint4 v = __ldcs(reinterpret_cast<const uint4 *>(a.y + static_cast<size_t>(rows[j]) * H) + c);
-      const __half2 *hv = reinterpret_cast<const __half2 *>(&v);
+    for (int j0 = 0; j0 <= k; j0 += U) {
+      uint4 v[U];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float2 f = __half22float2(hv[q]);
-        acc[2 * q] += f.x;
-        acc[2 * q + 1] += f.y;
+      for (int u = 0; u < U; ++u) {
+        const int j = j0 + u;
+        v[u] = make_uint4(0, 0, 0, 0);
+        if (j <= k && rows[j] >= 0)
+          v[u] = __ldcs(reinterpret_cast<const uint4 *>(a.y + static_cast<size_t>(rows[j]) * H) + c);
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int j = j0 + u;
+        if (j > k || rows[j] < 0) continue;
+        const __half2 *hv = reinterpret_cast<const __half2 *>(&v[u]);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 f = __half22float2(hv[q]);
+          acc[2 * q] += f.x;
+          acc[2 * q + 1] += f.y;
+        }
       }
     }
     uint4 res;
@@ -75,9 +91,12 @@ cudaError_t launch_host_stage(const HostStageArgs &a, cudaStream_t s, bool pdl) 
   return launch_k(host_stage_kernel, dim3(1), dim3(256), 0, s, pdl, a);
 }
 
+constexpr int kCombineFewTokens = 1024;  // at most this many tokens: rows requested nine at a time
+
 cudaError_t launch_combine(const CombineArgs &a, cudaStream_t s, bool pdl) {
   if (a.T <= 0) return cudaSuccess;
-  return launch_k(combine_kernel, dim3(a.T), dim3(256), 0, s, pdl, a);
+  if (a.T <= kCombineFewTokens) return launch_k(combine_kernel<9>, dim3(a.T), dim3(256), 0, s, pdl, a);
+  return launch_k(combine_kernel<1>, dim3(a.T), dim3(256), 0, s, pdl, a);
 }
 
 }  // namespace moe
