@@ -197,13 +197,14 @@ struct ProfScope {
 
 // routing kernels: ids/weights + histogram, scan + work lists, scatter, gather (if x)
 moe_status enqueue_routing(moe_plan_s *p, int T, const float *logits, const uint16_t *x, cudaStream_t s) {
-  const int nchunk = static_cast<int>(cdiv(T, kRouteChunk));
+  const int chunk = route_chunk(T);
+  const int nchunk = static_cast<int>(cdiv(T, chunk));
   // one warp per token, two per block: a few hundred tokens still spread over every SM
   const int tok_blocks = static_cast<int>(cdiv(T, 2));
   {
     ProfScope ps(p, MOE_KERNEL_ROUTE_TOPK, s);
-    MOE_CUDA(launch_k(route_topk_kernel, dim3(tok_blocks), dim3(64), 0, s, pdl(p), T, p->E, p->k, logits, p->ids,
-                      p->wts, p->chunk),
+    MOE_CUDA(launch_k(route_topk_kernel, dim3(tok_blocks), dim3(64), 0, s, pdl(p), T, p->E, p->k, chunk, logits,
+                      p->ids, p->wts, p->chunk),
              "route_topk launch");
   }
   RouteScanArgs sa{};
@@ -214,7 +215,7 @@ moe_status enqueue_routing(moe_plan_s *p, int T, const float *logits, const uint
              "route_scan launch");
   }
   RouteScatterArgs ca{};
-  ca.T = T; ca.E = p->E; ca.k = p->k; ca.H = p->H; ca.I = p->I; ca.Is = p->Is;
+  ca.T = T; ca.E = p->E; ca.k = p->k; ca.H = p->H; ca.I = p->I; ca.Is = p->Is; ca.chunk = chunk;
   ca.ids = p->ids; ca.chunk_base = p->chunk; ca.totals = p->totals; ca.offsets = p->offsets; ca.perm = p->perm;
   ca.inv = p->inv;
   ca.gu_items = p->gu_items; ca.max_gu = static_cast<int>(p->max_gu); ca.gu_tile = gu_tile_rows(T, p->k, p->E);
@@ -350,7 +351,7 @@ moe_status moe_plan(int T_max, int hidden, int n_experts, int top_k, int inter, 
   p->max_gu = max_gu_items_plan(T_max, n_experts, top_k, inter, shared_inter);
   p->max_dn = max_dn_items(T_max, n_experts, top_k, hidden);
   const size_t T = T_max, H = hidden, E = n_experts, k = top_k, I = inter, Is = shared_inter;
-  const size_t R = T * k, nchunk = (T + kRouteChunk - 1) / kRouteChunk;
+  const size_t R = T * k, nchunk = (T + kRouteChunkMin - 1) / kRouteChunkMin;  // the most chunks any batch has
   const size_t sizes[] = {
       R * 4,                                 // ids
       R * 4,                                 // wts

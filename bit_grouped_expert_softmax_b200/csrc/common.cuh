@@ -16,7 +16,16 @@ constexpr int kGroup = 64;       // weights per scale/bias group (along K)
 constexpr int kMaxExperts = 256; // one warp holds a token's logits in 8 registers per lane
 constexpr int kMaxTopK = 16;
 constexpr int kSmallT = 8;       // batches up to this size take the fused small-T kernel
-constexpr int kRouteChunk = 32;  // tokens per routing block
+constexpr int kRouteChunk = 32;     // tokens per routing block, at most
+constexpr int kRouteChunkMin = 8;   // ... and at least
+
+// Tokens per routing block for a batch of T: 8 while the batch is small
+// (more blocks share the scatter's serial ranking), 32 when it is large
+// (fewer chunk columns for the scan, fewer blocks repeating the offset scan);
+// measured at T = 512, 4096 and 8192.
+inline int route_chunk(int64_t T) {
+  return T <= 512 ? kRouteChunkMin : T <= 1024 ? 16 : kRouteChunk;
+}
 
 // Device status word: first error wins, later ones are dropped.
 enum DevError : uint32_t { kDevOk = 0, kDevTimeout = 1, kDevBounds = 2 };

@@ -28,6 +28,7 @@ struct RouteScanArgs {
 
 struct RouteScatterArgs {
   int T, E, k, H, I, Is;
+  int chunk;                  // tokens per routing chunk (one scatter block each)
   const int32_t *ids;         // [T*k]
   int32_t *chunk_base;        // [nchunk][E] per-chunk prefixes in; zeroed on the way out
   const int32_t *totals;      // [E] rows routed to each expert
@@ -135,7 +136,7 @@ struct RouterArgs {
   DevStatus *status;
 };
 
-__global__ void route_topk_kernel(int T, int E, int k, const float *__restrict__ logits,
+__global__ void route_topk_kernel(int T, int E, int k, int chunk, const float *__restrict__ logits,
                                   int32_t *__restrict__ ids, float *__restrict__ wts,
                                   int32_t *__restrict__ chunk_cnt);
 __global__ void route_scan_kernel(RouteScanArgs a);

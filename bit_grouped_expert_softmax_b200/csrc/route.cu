@@ -24,7 +24,7 @@
 
 namespace moe {
 
-__global__ void __launch_bounds__(256) route_topk_kernel(int T, int E, int k,
+__global__ void __launch_bounds__(256) route_topk_kernel(int T, int E, int k, int chunk,
                                                          const float *__restrict__ logits,
                                                          int32_t *__restrict__ ids,
                                                          float *__restrict__ wts,
@@ -42,7 +42,7 @@ __global__ void __launch_bounds__(256) route_topk_kernel(int T, int E, int k,
   if (lane < k) {
     ids[static_cast<size_t>(t) * k + lane] = id;
     wts[static_cast<size_t>(t) * k + lane] = w;
-    atomicAdd(&chunk_cnt[static_cast<size_t>(t / kRouteChunk) * E + id], 1);
+    atomicAdd(&chunk_cnt[static_cast<size_t>(t / chunk) * E + id], 1);
   }
 }
 
@@ -97,7 +97,7 @@ __global__ void __launch_bounds__(256) route_scatter_kernel(RouteScatterArgs a) 
   const int G = E + 1;  // routed experts plus the shared one
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int32_t *row = a.chunk_base + static_cast<size_t>(chunk) * E;
-  const int t0 = chunk * kRouteChunk, t1 = min(T, t0 + kRouteChunk);
+  const int t0 = chunk * a.chunk, t1 = min(T, t0 + a.chunk);
   const int f0 = t0 * k, f1 = t1 * k;
   // the experts' totals, the chunk's per-expert prefix and the chunk's ids,
   // all loaded by the whole block at once
