@@ -71,6 +71,20 @@ struct TmaRing {
   __device__ __forceinline__ void drain(uint64_t *full) const { drain_stages<N>(full, issued, issued_ph); }
 };
 
+// The consumer side of an N-stage ring: the stage index and the parity of its
+// current phase.
+template <int N>
+struct RingCursor {
+  int s = 0;
+  uint32_t ph = 0;
+  __device__ __forceinline__ void advance() {
+    if (++s == N) {
+      s = 0;
+      ph ^= 1u;
+    }
+  }
+};
+
 // Whether a work item lies inside the buffers it addresses: its expert, its
 // 128-row weight block and its activation rows (routed rows in [0, R), the
 // shared expert's rows in [R, R + T)); every TMA coordinate of the item
@@ -131,6 +145,35 @@ __device__ __forceinline__ uint16_t pick_bf16(uint2 v, int j) {
   const uint32_t w = (j & 2) ? v.y : v.x;
   return static_cast<uint16_t>((j & 1) ? w >> 16 : w);
 }
+
+// The scales and biases of one weight row as the dequantisation walks its
+// K-blocks: four K-blocks per load, one packed stage ahead, and during the
+// last packed stage of an item the first four of the next item's row.
+struct SbStream {
+  SbRow row{}, next{};
+  uint2 s_cur{}, b_cur{}, s_nxt{}, b_nxt{};
+
+  __device__ __forceinline__ void start(const SbRow &r) {
+    row = next = r;
+    load_sb4(row, 0, s_nxt, b_nxt);
+  }
+  // At K-block kb (a multiple of 4) of a row of nkb K-blocks: K-blocks kb ..
+  // kb + 3 become current and the next four are requested; next_row(r) gives
+  // the next item's row (returns false if there is none).
+  template <class NextRow>
+  __device__ __forceinline__ void step(int kb, int nkb, NextRow next_row) {
+    s_cur = s_nxt;
+    b_cur = b_nxt;
+    if (kb + 4 < nkb) {
+      load_sb4(row, kb + 4, s_nxt, b_nxt);
+    } else if (next_row(next)) {
+      load_sb4(next, 0, s_nxt, b_nxt);
+    }
+  }
+  __device__ __forceinline__ void end_item() { row = next; }
+  __device__ __forceinline__ __half2 scale(int j) const { return bf16_to_half2_bcast(pick_bf16(s_cur, j)); }
+  __device__ __forceinline__ __half2 bias(int j) const { return bf16_to_half2_bcast(pick_bf16(b_cur, j)); }
+};
 
 // Dequantise two packed words (16 weights of one row) into 8 fp16 pairs.
 __device__ __forceinline__ void dequant2(uint32_t w0, uint32_t w1, __half2 s2, __half2 b2, uint32_t (&d)[8]) {

@@ -233,8 +233,8 @@ __global__ void __launch_bounds__(GuTile<N>::kThreads, 1) gemm_gate_up_kernel(co
     }
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------ MMA issuer (whole warp, one elected lane issues)
-    int sb = 0, sa = 0;
-    uint32_t phb = 0, pha = 0;
+    RingCursor<kBStages> bs;
+    RingCursor<kAStages> as;
     bool ok = true;
     int li = 0;
     for (int it = next_item(a, blockIdx.x, nitems, false, false); it < nitems && ok;
@@ -244,12 +244,12 @@ __global__ void __launch_bounds__(GuTile<N>::kThreads, 1) gemm_gate_up_kernel(co
       tc_fence_after();
       const uint32_t idesc = idesc_f16_f32(kRows, (wi.nrows + 15) & ~15);
       for (int ks = 0; ks < nkb / kStageK; ++ks) {
-        if (!warp_wait(&b_full[sb], phb, abort, a.status, 212)) {
+        if (!warp_wait(&b_full[bs.s], bs.ph, abort, a.status, 212)) {
           ok = false;
           break;
         }
-        const uint32_t b_addr = smem_u32(sB + sb * kBStageBytes);
-        if (!warp_wait(&a_full[sa], pha, abort, a.status, 211)) {
+        const uint32_t b_addr = smem_u32(sB + bs.s * kBStageBytes);
+        if (!warp_wait(&a_full[as.s], as.ph, abort, a.status, 211)) {
           ok = false;
           break;
         }
@@ -257,7 +257,7 @@ __global__ void __launch_bounds__(GuTile<N>::kThreads, 1) gemm_gate_up_kernel(co
         if (elect_one()) {
 #pragma unroll
           for (int kh = 0; kh < kStageK; ++kh) {
-            const uint32_t a_col = tmem_base + kACol0 + sa * kAStageCols + kh * 64;
+            const uint32_t a_col = tmem_base + kACol0 + as.s * kAStageCols + kh * 64;
 #pragma unroll
             for (int kk = 0; kk < kTileK / 16; ++kk) {
               const uint64_t bdesc = smem_desc_sw128(b_addr + kh * kBAtomBytes + kk * 32);
@@ -266,18 +266,12 @@ __global__ void __launch_bounds__(GuTile<N>::kThreads, 1) gemm_gate_up_kernel(co
               tc_mma_f16_ts(tmem_base + kAccCols, a_col + 32 + kk * 8, bdesc, idesc, acc);
             }
           }
-          tc_commit(&a_empty[sa]);
-          tc_commit(&b_empty[sb]);
+          tc_commit(&a_empty[as.s]);
+          tc_commit(&b_empty[bs.s]);
         }
         __syncwarp();
-        if (++sa == kAStages) {
-          sa = 0;
-          pha ^= 1u;
-        }
-        if (++sb == kBStages) {
-          sb = 0;
-          phb ^= 1u;
-        }
+        as.advance();
+        bs.advance();
       }
       if (ok && elect_one()) tc_commit(acc_full);
       __syncwarp();
@@ -380,44 +374,32 @@ __global__ void __launch_bounds__(GuTile<N>::kThreads, 1) gemm_gate_up_kernel(co
     const int r = q * 32 + lane;
     const int m = (dw >> 2) & 1;  // 0: gate, 1: up
     const int half = dw >> 3;     // 0 unless kDqPerQ == 2
-    int sp = 0, sa = 0;
-    uint32_t php = 0, pha = 0;
+    RingCursor<kPkStages> pk;
+    RingCursor<kAStages> as;
     bool ok = true;
-    // scales and biases: four K-blocks per load, one packed stage ahead; the
-    // first stage of the next item is fetched during the last stage of this one
-    SbRow row{};
-    uint2 s_cur{}, b_cur{}, s_nxt{}, b_nxt{};
+    static_assert(kSuperK == 4, "the scale/bias stream loads four K-blocks at a time");
+    SbStream sb;
     const int first = next_item(a, blockIdx.x, nitems, false, false);
-    if (first < nitems) {
-      row = sb_row_gu(a, a.items[first], m, r);
-      load_sb4(row, 0, s_nxt, b_nxt);
-    }
+    if (first < nitems) sb.start(sb_row_gu(a, a.items[first], m, r));
     for (int it = first; it < nitems && ok; it = next_item(a, it + gridDim.x, nitems, false, false)) {
-      SbRow next_row = row;
       for (int kb = 0; kb < nkb; kb += kAKB) {  // two K-blocks per TMEM stage
         const int j = kb % kSuperK;             // 0 or 2 within the packed stage
-        if (j == 0) {
-          s_cur = s_nxt;
-          b_cur = b_nxt;
-          if (kb + kSuperK < nkb) {
-            load_sb4(row, kb + kSuperK, s_nxt, b_nxt);
-          } else if (const int nx = next_item(a, it + gridDim.x, nitems, false, false); nx < nitems) {
-            next_row = sb_row_gu(a, a.items[nx], m, r);
-            load_sb4(next_row, 0, s_nxt, b_nxt);
-          }
-        }
-        const __half2 s2a = bf16_to_half2_bcast(pick_bf16(s_cur, j));
-        const __half2 b2a = bf16_to_half2_bcast(pick_bf16(b_cur, j));
-        const __half2 s2b = bf16_to_half2_bcast(pick_bf16(s_cur, j + 1));
-        const __half2 b2b = bf16_to_half2_bcast(pick_bf16(b_cur, j + 1));
-        if (j == 0 && !warp_wait(&pk_full[sp], php, abort, a.status, 230)) {
+        if (j == 0)
+          sb.step(kb, nkb, [&](SbRow &nr) {
+            const int nx = next_item(a, it + gridDim.x, nitems, false, false);
+            if (nx >= nitems) return false;
+            nr = sb_row_gu(a, a.items[nx], m, r);
+            return true;
+          });
+        const __half2 s2a = sb.scale(j), b2a = sb.bias(j), s2b = sb.scale(j + 1), b2b = sb.bias(j + 1);
+        if (j == 0 && !warp_wait(&pk_full[pk.s], pk.ph, abort, a.status, 230)) {
           ok = false;
           break;
         }
         // row r of the packed tile: 128 bytes = 4 K-blocks of 8 words, in
         // 16-byte chunks placed at chunk ^ (r & 7) by the TMA's 128-byte swizzle;
         // chunk c of K-block j + kk is 2 (j + kk) + c
-        const uint8_t *prow = sPk + sp * kPkStageBytes + m * kPkTileBytes + r * 128;
+        const uint8_t *prow = sPk + pk.s * kPkStageBytes + m * kPkTileBytes + r * 128;
         uint4 v[2][kCh];
 #pragma unroll
         for (int kk = 0; kk < 2; ++kk)
@@ -426,20 +408,17 @@ __global__ void __launch_bounds__(GuTile<N>::kThreads, 1) gemm_gate_up_kernel(co
             v[kk][c] = *reinterpret_cast<const uint4 *>(prow + (((2 * (j + kk) + c * kDqPerQ + half) ^ (r & 7)) << 4));
         if (j + kAKB == kSuperK || kb + kAKB >= nkb) {  // words in registers: release the packed stage
           __syncwarp();
-          if (lane == 0) mbar_arrive(&pk_empty[sp]);
-          if (++sp == kPkStages) {
-            sp = 0;
-            php ^= 1u;
-          }
+          if (lane == 0) mbar_arrive(&pk_empty[pk.s]);
+          pk.advance();
         }
         // pieces of 8 columns whose stores overlap the next piece's
         // arithmetic; the first is computed before the stage is known free;
         // one wait. Chunk c of a K-block fills columns 16 c .. 16 c + 15 of
         // the matrix's 32 in that K-block's 64.
-        const uint32_t ta = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + kACol0 + sa * kAStageCols + m * 32;
+        const uint32_t ta = tmem_base + (static_cast<uint32_t>(q * 32) << 16) + kACol0 + as.s * kAStageCols + m * 32;
         uint32_t d8[8];
         dequant2(v[0][0].x, v[0][0].y, s2a, b2a, d8);
-        if (!warp_wait(&a_empty[sa], pha ^ 1u, abort, a.status, 231)) {
+        if (!warp_wait(&a_empty[as.s], as.ph ^ 1u, abort, a.status, 231)) {
           ok = false;
           break;
         }
@@ -456,13 +435,10 @@ __global__ void __launch_bounds__(GuTile<N>::kThreads, 1) gemm_gate_up_kernel(co
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&a_full[sa]);
-        if (++sa == kAStages) {
-          sa = 0;
-          pha ^= 1u;
-        }
+        if (lane == 0) mbar_arrive(&a_full[as.s]);
+        as.advance();
       }
-      row = next_row;
+      sb.end_item();
     }
     }
   }
