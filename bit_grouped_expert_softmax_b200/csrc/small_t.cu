@@ -7,29 +7,34 @@
 //
 //   entry    the shared expert needs no routing: each CTA requests, with bulk
 //            asynchronous copies into shared memory, its shared-expert gate/up
-//            row block and the shared expert's down rows of its output slice
-//            before it looks at a logit
+//            row block and the shared expert's down rows of its output slice,
+//            before it waits for the kernel ahead on the stream (programmatic
+//            dependent launch) and before it looks at a logit
 //   routing  every CTA routes the (<= 8) tokens itself (same result in every
-//            CTA) with all its warps: each warp takes the top k of one 32-expert
-//            slice of one token, then one warp per token merges the slices'
-//            candidates; the distinct experts are listed and their gate/up row
-//            blocks and down rows requested at once, from several warps
+//            CTA) with all its warps: each warp ranks the logits of one
+//            32-expert slice of one token by shuffles and keeps that slice's
+//            top k, then one thread per candidate counts the candidates that
+//            precede it; the distinct experts are listed and their gate/up
+//            row blocks requested from several warps at once, their down rows
+//            right after
 //   gate/up  each 16-row block of an expert is split along K over several
 //            warps; tensor-core mma.sync m16n8k16 with A = dequantised weights
 //            (fp16 q*scale+bias, as in the grouped GEMM) and B = the tokens
-//            (N = 8 covers every token at once); partial sums reduced in a fixed
-//            order, h = silu(gate) * up written to a small scratch, and the
-//            expert's readiness counter incremented (release)
+//            (N = 8 covers every token at once); the partial sums are reduced
+//            in a fixed order by up to four warps, each of which writes its
+//            part of h = silu(gate) * up to a small scratch and increments the
+//            expert's readiness counter (release)
 //   down     each CTA owns 16 output features; warp w takes the used experts
 //            u = w, w + 16, ...; it waits (bounded, acquire) until every row
 //            block of expert u has published its h, then multiplies that h by
 //            the down rows already in shared memory and weights each token's
 //            result by its routing weight; the warps' results are summed in a
 //            fixed order and rounded once
-//   exit     once all its warps are past their last counter poll, a CTA counts
-//            itself out; the CTA that completes the count clears the counters
-//            for the next launch on the stream. A CTA that gave up on a wait
-//            waits for its own copies still in flight before it leaves
+//   exit     once all its warps are past their last counter poll, a CTA adds
+//            itself to an exit count (release increment); a warp of CTA 0
+//            waits for the full count and clears the counters for the next
+//            launch on the stream. A CTA that gave up on a wait waits for its
+//            own copies still in flight before it leaves
 //
 // There is no grid-wide barrier: an expert's down product starts as soon as
 // that expert's h is complete, while other experts' gate/up blocks finish.
