@@ -97,7 +97,7 @@ struct moe_plan_s {
   __half *xt;
   __half *h;
   __half *y;
-  __half *hsmall;
+  uint64_t *hsmall;  // small-T SwiGLU outputs (tagged fp16 pairs)
   DevStatus *status;
   uint32_t *small_sync;
   uint16_t *x_stage;
@@ -369,9 +369,9 @@ moe_status moe_plan(int T_max, int hidden, int n_experts, int top_k, int inter, 
       (R + T) * H * 2,                       // xt
       (R * I + T * Is) * 2,                  // h
       (R + T) * H * 2,                       // y
-      static_cast<size_t>(kSmallT) * (k + 1) * std::max(I, Is) * 2,  // small-T h (fp16)
+      static_cast<size_t>(kSmallT) * (k + 1) * std::max(I, Is) * 4,  // small-T h (tagged fp16 pairs)
       sizeof(DevStatus),                     // status
-      kSmallTSyncWords * 4,                  // small-T readiness and exit counters
+      kSmallTSyncWords * 4,                  // small-T counters and launch tag
       T * H * 2,                             // x staging
       T * E * 4,                             // logits staging
       T * E * 4,                             // router scores
@@ -407,7 +407,7 @@ moe_status moe_plan(int T_max, int hidden, int n_experts, int top_k, int inter, 
   p->xt = reinterpret_cast<__half *>(b + offs[i++]);
   p->h = reinterpret_cast<__half *>(b + offs[i++]);
   p->y = reinterpret_cast<__half *>(b + offs[i++]);
-  p->hsmall = reinterpret_cast<__half *>(b + offs[i++]);
+  p->hsmall = reinterpret_cast<uint64_t *>(b + offs[i++]);
   p->status = reinterpret_cast<DevStatus *>(b + offs[i++]);
   p->small_sync = reinterpret_cast<uint32_t *>(b + offs[i++]);
   p->x_stage = reinterpret_cast<uint16_t *>(b + offs[i++]);
@@ -703,8 +703,9 @@ moe_status moe_status_sync(moe_plan_t *plan, moe_stream_t stream) {
   MOE_CUDA(cudaMemcpy(&h, plan->status, sizeof h, cudaMemcpyDeviceToHost), "read status");
   if (h.code == kDevOk) return MOE_OK;
   // clear the status and the small-T counters so the plan can be used again
+  // (the small-T launch tag is kept: a later launch must not reuse it)
   MOE_CUDA(cudaMemset(plan->status, 0, sizeof(DevStatus)), "clear status");
-  MOE_CUDA(cudaMemset(plan->small_sync, 0, kSmallTSyncWords * 4), "clear small-T counters");
+  MOE_CUDA(cudaMemset(plan->small_sync, 0, kSmallTCounterWords * 4), "clear small-T counters");
   MOE_CUDA(cudaDeviceSynchronize(), "synchronize");
   if (h.code == kDevTimeout)
     return fail(MOE_ERR_DEVICE_TIMEOUT, "device wait ran out (site %u, block %u)", h.where, h.detail);

@@ -97,10 +97,15 @@ struct CombineArgs {
 
 // Distinct experts one small-T launch can use: the shared one plus T*k routed.
 constexpr int kSmallTMaxU = kSmallT * kMaxTopK + 1;
-// Synchronisation words of the small-T kernel: one readiness counter per used
-// expert, the exit counter, then the count of CTAs whose router scores are
-// published. They must be zero before a launch; each launch leaves them zero.
-constexpr int kSmallTSyncWords = kSmallTMaxU + 2;
+// Synchronisation words of the small-T kernel: the exit count and the count of
+// CTAs whose router scores are published (zero before a launch; each launch
+// leaves them zero), then the tag of the last launch (zero in a new buffer;
+// kept across launches, never cleared).
+constexpr int kSmallTExitWord = 0;
+constexpr int kSmallTRouterWord = 1;
+constexpr int kSmallTEpochWord = 2;
+constexpr int kSmallTCounterWords = 2;  // the words a recovery clears
+constexpr int kSmallTSyncWords = 3;
 
 struct SmallTArgs {
   int T, E, k, H, I, Is;
@@ -108,8 +113,9 @@ struct SmallTArgs {
   const float *logits;      // [T, E]; written by the kernel itself when router_w is set
   const uint16_t *router_w; // [E, H] bf16 router weight, or null (logits given)
   LayerWeights w;
-  __half *hbuf;             // [8][k+1][max(I,Is)] fp16 scratch: SwiGLU outputs by token and slot
-  uint32_t *sync;           // [kSmallTSyncWords] readiness and exit counters (zero between launches)
+  uint64_t *hbuf;           // [8][k+1][max(I,Is)/2] SwiGLU outputs by token and slot: two fp16 values and
+                            // the launch tag per word (cleared to zero before the first launch)
+  uint32_t *sync;           // [kSmallTSyncWords] exit and router counters, last launch tag
   const uint16_t *residual; // [T, H] or null
   uint16_t *out;            // [T, H]
   DevStatus *status;

@@ -27,15 +27,18 @@ using namespace moe;
 namespace {
 
 constexpr size_t kStaticScratchBytes = 512 * 1024;  // stated maximum
-constexpr size_t kSyncOff = 0;                      // readiness and exit counters of the kernel
+constexpr size_t kSyncOff = 0;                      // the kernel's counters, then its launch tag
 constexpr size_t kStatusOff = 1024;                 // DevStatus
-constexpr size_t kHeaderBytes = 1280;               // cleared before every launch
-constexpr size_t kHOff = kHeaderBytes;              // fp16 SwiGLU outputs, 8 * (top_k + 1) * max(I, Is)
+constexpr size_t kHeaderBytes = 1280;
+constexpr size_t kHOff = kHeaderBytes;              // SwiGLU outputs, 8 * (top_k + 1) * max(I, Is) tagged values
 constexpr int kMaxDevices = 64;
 static_assert(kSmallTSyncWords * 4 <= kStatusOff - kSyncOff, "counters fit the header");
 
-// [0, 1024): the kernel's synchronisation counters; [1024, 1040): DevStatus;
-// [1280, kStaticScratchBytes): fp16 SwiGLU outputs by token and slot.
+// [0, 12): the kernel's exit and router counters (cleared before every
+// launch) and its last launch tag (kept: a launch must not reuse the tag of
+// one before it); [1024, 1040): DevStatus (cleared before every launch);
+// [1280, kStaticScratchBytes): SwiGLU outputs by token and slot as 8-byte
+// words of two fp16 values and a launch tag (zero-initialised with the module).
 static __device__ __align__(256) unsigned char g_small_t_scratch[kStaticScratchBytes];
 
 struct DeviceSlot {
@@ -91,9 +94,9 @@ extern "C" moe_status moe_forward_small_t_noalloc(int T, int hidden, int n_exper
   if (n_experts < 1 || n_experts > kMaxExperts || top_k < 1 || top_k > n_experts || top_k > kMaxTopK)
     return fail(MOE_ERR_INVALID_ARG, "need 1 <= top_k <= min(n_experts, 16) and n_experts <= 256");
   const size_t imax = static_cast<size_t>(inter > shared_inter ? inter : shared_inter);
-  const size_t h_bytes = static_cast<size_t>(kSmallT) * (top_k + 1) * imax * sizeof(__half);
+  const size_t h_bytes = static_cast<size_t>(kSmallT) * (top_k + 1) * imax * 4;  // a tagged word per 2 values
   if (kHOff + h_bytes > kStaticScratchBytes)
-    return fail(MOE_ERR_UNSUPPORTED, "8 * (top_k + 1) * max(inter, shared_inter) * 2 bytes exceeds the 512 KiB "
+    return fail(MOE_ERR_UNSUPPORTED, "8 * (top_k + 1) * max(inter, shared_inter) * 4 bytes exceeds the 512 KiB "
                                      "static scratch (less its 1280-byte header)");
   if (status_out && (reinterpret_cast<uintptr_t>(status_out) & 15u))
     return fail(MOE_ERR_INVALID_ARG, "status_out must be 16-byte aligned");
@@ -120,8 +123,10 @@ extern "C" moe_status moe_forward_small_t_noalloc(int T, int hidden, int n_exper
   if (!small_t_fits(T, hidden, top_k, inter, shared_inter, slot->num_sms))
     return fail(MOE_ERR_UNSUPPORTED, "layer too large for the small-T kernel (shared memory or hidden/16 > SMs)");
 
-  // the array keeps the previous call's contents: clear the counters and the status word
-  err = cudaMemsetAsync(slot->ptr, 0, kHeaderBytes, s);
+  // the array keeps the previous call's contents: clear the counters and the
+  // status word (the launch tag stays)
+  err = cudaMemsetAsync(slot->ptr + kSyncOff, 0, kSmallTCounterWords * 4, s);
+  if (err == cudaSuccess) err = cudaMemsetAsync(slot->ptr + kStatusOff, 0, sizeof(DevStatus), s);
   if (err != cudaSuccess) return fail(MOE_ERR_CUDA, "clearing the static scratch header failed");
   SmallTArgs a{};  // value-initialised: every field not set below is zero (no router: logits are given)
   a.T = T; a.E = n_experts; a.k = top_k; a.H = hidden; a.I = inter; a.Is = shared_inter;
@@ -136,7 +141,7 @@ extern "C" moe_status moe_forward_small_t_noalloc(int T, int hidden, int n_exper
   a.w.sh_biases = static_cast<const uint16_t *>(shared_biases);
   a.sync = reinterpret_cast<uint32_t *>(slot->ptr + kSyncOff);
   a.status = reinterpret_cast<DevStatus *>(slot->ptr + kStatusOff);
-  a.hbuf = reinterpret_cast<__half *>(slot->ptr + kHOff);
+  a.hbuf = reinterpret_cast<uint64_t *>(slot->ptr + kHOff);
   a.residual = nullptr;
   a.out = static_cast<uint16_t *>(out_bf16);
   a.wait_ns = kWaitBudgetNs;

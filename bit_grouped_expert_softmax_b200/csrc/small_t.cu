@@ -21,23 +21,24 @@
 //            warps; tensor-core mma.sync m16n8k16 with A = dequantised weights
 //            (fp16 q*scale+bias, as in the grouped GEMM) and B = the tokens
 //            (N = 8 covers every token at once); the partial sums are reduced
-//            in a fixed order by up to four warps, each of which writes its
-//            part of h = silu(gate) * up to a small scratch and increments the
-//            expert's readiness counter (release)
+//            in a fixed order by up to four warps, each of which stores its
+//            part of h = silu(gate) * up to a small scratch as tagged words
+//            (two fp16 values and the launch tag in one 8-byte store)
 //   down     each CTA owns 16 output features; warp w takes the used experts
-//            u = w, w + 16, ...; it waits (bounded, acquire) until every row
-//            block of expert u has published its h, then multiplies that h by
-//            the down rows already in shared memory and weights each token's
+//            u = w, w + 16, ...; it reads expert u's h (bounded polling, until
+//            every word carries this launch's tag), then multiplies it by the
+//            down rows already in shared memory and weights each token's
 //            result by its routing weight; the warps' results are summed in a
 //            fixed order and rounded once
-//   exit     once all its warps are past their last counter poll, a CTA adds
-//            itself to an exit count (release increment); a warp of CTA 0
-//            waits for the full count and clears the counters for the next
-//            launch on the stream. A CTA that gave up on a wait waits for its
-//            own copies still in flight before it leaves
+//   exit     every CTA adds itself to an exit count (release increment) once it
+//            has read the launch tag; a warp of CTA 0 waits for the full count,
+//            clears the counters and records the tag for the next launch on
+//            the stream. A CTA that gave up on a wait waits for its own copies
+//            still in flight before it leaves
 //
-// There is no grid-wide barrier: an expert's down product starts as soon as
-// that expert's h is complete, while other experts' gate/up blocks finish.
+// There is no grid-wide barrier and no readiness counter: an expert's down
+// product starts as soon as that expert's h words have all arrived, while
+// other experts' gate/up blocks finish.
 //
 // Operand order along K: packed word W holds elements 8W..8W+7; the fp16
 // operands store them at positions 8W + s in the pair order (0,4),(1,5),(2,6),
@@ -66,6 +67,7 @@ constexpr int kSlices = kMaxExperts / 32;  // 32-expert slices of a token's logi
 constexpr int kCandPerToken = kSlices * kMaxTopK;  // routing candidates of one token, at most
 static_assert(kSmallTMaxU == kSmallT * kMaxTopK + 1, "one shared plus at most T*k routed experts");
 constexpr int kMaxU = kSmallTMaxU;
+constexpr int kPairsPerLane = 4;  // staged poll of tagged h words: at most 128 pairs per expert
 
 struct SmallTShared {
   int ids[kSmallT][kMaxTopK];
@@ -79,7 +81,7 @@ struct SmallTShared {
   int b_iss[4];                        // copies issued into each phase-1 stage
   int d_iss[kMaxU];                    // copies issued into each phase-2 stage
   int nU;
-  int polled;  // warps done reading readiness counters
+  uint32_t tag;  // this launch's tag of the SwiGLU output words
   int abort;
 };
 
@@ -185,6 +187,29 @@ __device__ __forceinline__ void drain_ring(uint64_t *full, const int *issued, in
   }
 }
 
+// The SwiGLU outputs go from the CTAs that compute them to the CTAs that
+// multiply them by the down rows as 8-byte words: two fp16 values (K positions
+// 2w, 2w + 1) in the low half and the launch's tag in the high half. A naturally
+// aligned 8-byte store or load is single-copy atomic, so a reader that sees
+// the tag also sees the values stored with it: no fence, no counter and no
+// second read are needed between the two sides. The tag changes every launch
+// and is never 0 (the value the scratch is cleared to).
+__device__ __forceinline__ void st_tagged(uint64_t *p, uint64_t v) {
+  asm volatile("st.relaxed.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+__device__ __forceinline__ ulonglong2 ld_tagged2(const uint64_t *p) {
+  ulonglong2 r;
+  asm volatile("ld.relaxed.gpu.global.v2.u64 {%0, %1}, [%2];" : "=l"(r.x), "=l"(r.y) : "l"(p) : "memory");
+  return r;
+}
+__device__ __forceinline__ bool tag_ok(const ulonglong2 &v, uint32_t tag) {
+  return static_cast<uint32_t>(v.x >> 32) == tag && static_cast<uint32_t>(v.y >> 32) == tag;
+}
+// the four fp16 values of a word pair
+__device__ __forceinline__ uint2 tagged_values(const ulonglong2 &v) {
+  return make_uint2(static_cast<uint32_t>(v.x), static_cast<uint32_t>(v.y));
+}
+
 __device__ __forceinline__ void bulk_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
                    smem_u32(dst)),
@@ -281,10 +306,9 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs
   uint64_t *b_full = reinterpret_cast<uint64_t *>(dyn + L.bar_off);
   uint64_t *d_full = b_full + L.nb;
   volatile int *abort = &sh.abort;
-  __half *hb = a.hbuf;                               // [T][k+1][Imax] fp16 scratch, operand order
-  uint32_t *ready = a.sync;                          // [kMaxU] readiness counters
-  uint32_t *exit_count = a.sync + kMaxU;
-  uint32_t *router_count = a.sync + kMaxU + 1;       // CTAs whose router scores are published
+  uint64_t *hb = a.hbuf;                             // [T][k+1][Imax/2] tagged words, operand order
+  uint32_t *exit_count = a.sync + kSmallTExitWord;
+  uint32_t *router_count = a.sync + kSmallTRouterWord;  // CTAs whose router scores are published
   const unsigned long long budget = a.wait_ns;
   const int Imax = L.Imax;
   const int nrb_sh = a.Is / kRowBlock;               // the shared expert's row blocks: the first units
@@ -297,7 +321,6 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs
   if (threadIdx.x == 0) {
     for (int s = 0; s < L.nb + L.nd; ++s) mbar_init(&b_full[s], 1);
     sh.abort = 0;
-    sh.polled = 0;
     sh.ulist[0] = E;
     fence_barrier_init();
     fence_proxy_async_smem();
@@ -388,6 +411,13 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs
   if (warp == 0 && shared_first) issue_b(0);
   if (warp == 1 && has_dblk) issue_d_range(0, 1);  // expert u = 0 is the shared one
   pdl_wait();
+  // this launch's tag: one more than the last launch's (0 skipped); the word is
+  // written only by the last step of a launch, once every CTA has read it
+  if (threadIdx.x == 0) {
+    uint32_t e;
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(e) : "l"(a.sync + kSmallTEpochWord) : "memory");
+    sh.tag = e + 1 == 0 ? 1u : e + 1;
+  }
   // every CTA of this grid is resident once all have passed here, so the next
   // launch's CTAs, which take SMs only as this grid's leave, cannot keep one
   // of them waiting
@@ -493,6 +523,9 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs
     if (lane == 0 && idx0 < nxc && m > 0.f) atomicMax(&sh.xexp[idx0 / hw], __float_as_int(m));
   }
   __syncthreads();
+  // this CTA has read the launch tag and is past the router-score wait: it
+  // reads neither counter again (the release orders the tag read before it)
+  if (threadIdx.x == 0) asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(exit_count) : "memory");
 
   // ---- routing, step 2: the token's top k among its slices' candidates --------------------
   // The token's top k lie among the slices' top k. One thread per candidate
@@ -677,18 +710,18 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs
           U += zp[4 + i];
         }
         const int t = 2 * c + (i & 1);
-        const int row = rb * kRowBlock + g + (i >> 1) * 8;
-        if (t < T && ((sh.umask[u] >> t) & 1u)) {
+        const int row0 = rb * kRowBlock + (i >> 1) * 8;  // this element's 8-row group; the lane's row is row0 + g
+        const bool mine = t < T && ((sh.umask[u] >> t) & 1u);
+        const uint32_t hbits = mine ? __half_as_ushort(__float2half_rn(swiglu_scaled(G, U, sh.xexp[t]))) : 0u;
+        // K positions 2g and 2g + 1 of the group hold rows g and g + 4 (the
+        // operand order), which lanes g and g + 4 of the same column computed
+        const uint32_t hi = __shfl_xor_sync(0xffffffffu, hbits, 16);
+        if (g < 4 && mine && !(a.test_fault && unit == 0)) {
           const int j = sh.uslot[u][t];
-          const float hv = swiglu_scaled(G, U, sh.xexp[t]);
-          hb[(static_cast<size_t>(t) * (k + 1) + j) * Imax + (row & ~7) + kperm_dst(row & 7)] = __float2half_rn(hv);
+          st_tagged(hb + (static_cast<size_t>(t) * (k + 1) + j) * (Imax / 2) + row0 / 2 + g,
+                    (static_cast<uint64_t>(sh.tag) << 32) | (hi << 16) | hbits);
         }
       }
-      // publish: the warp barrier orders every lane's h stores before lane 0's
-      // release increment, so a reader that acquires the count sees them
-      __syncwarp();
-      if (lane == 0 && !(a.test_fault && unit == 0))
-        asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(ready + u) : "memory");
     }
     __syncthreads();
     // the stages this round used are free: refill them with the units nb ahead
@@ -700,46 +733,55 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs
   }
 
   // ---- down + combine ----------------------------------------------------------------
-  // Each CTA adds itself to the exit count (a release increment, nothing to
-  // wait for) once all its warps are done reading readiness counters (a warp
-  // is done after its last poll, or at once if it has no expert to multiply).
-  // The last warp of CTA 0 then waits (bounded, acquire) for the whole grid's
-  // count and clears every counter for the next launch, which no CTA reads
-  // any more: off the critical path when that warp has no expert of its own,
-  // otherwise after its down products.
-  auto polls_done = [&]() {  // whole warp, once per warp
-    int last = 0;
-    if (lane == 0) last = atomicAdd(&sh.polled, 1) == kSTWarps - 1;
-    if (lane == 0 && last) asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(exit_count) : "memory");
+  // Every CTA counted itself out (exit count) once it had read the launch tag
+  // and was past the router-score wait. The last warp of CTA 0 waits
+  // (bounded, acquire) for the whole grid's count, clears the two counters and
+  // records the tag for the next launch, which no CTA of this one reads any
+  // more: off the critical path when that warp has no expert of its own,
+  // otherwise after its down products. The tag is recorded even when the wait
+  // runs out, so the next launch never reuses it.
+  const bool clears = blockIdx.x == 0 && warp == kSTWarps - 1;
+  auto clear_counters = [&]() {  // whole warp (CTA 0's last)
+    if (wait_count(exit_count, gridDim.x, abort, a.status, 44, 0, budget)) {
+      if (lane == kSmallTExitWord || lane == kSmallTRouterWord) a.sync[lane] = 0u;
+    }
+    if (lane == 0) asm volatile("st.relaxed.gpu.global.u32 [%0], %1;" ::"l"(a.sync + kSmallTEpochWord), "r"(sh.tag)
+                                : "memory");
     __syncwarp();
   };
-  const bool clears = blockIdx.x == 0 && warp == kSTWarps - 1;
-  auto clear_counters = [&]() {  // whole warp (CTA 0's last), after its own polls_done
-    if (wait_count(exit_count, gridDim.x, abort, a.status, 44, 0, budget)) {
-      for (int i = lane; i < kSmallTSyncWords; i += 32) a.sync[i] = 0u;
-    }
-  };
-  if (!has_dblk) {
-    polls_done();
-    if (clears) clear_counters();
-  }
+  if (!has_dblk && clears) clear_counters();
   if (has_dblk) {
     const int n0 = blockIdx.x * kRowBlock;
-    // each warp's share of the token staging area, for copies of h rows
+    const uint32_t tag = sh.tag;
+    // each warp's share of the token staging area, for the values of h rows
     const size_t h_slice_bytes = (L.red_off / kSTWarps) & ~static_cast<size_t>(15);
     float acc[4] = {0.f, 0.f, 0.f, 0.f};  // rows g, g+8; tokens 2c, 2c+1 (this warp's experts, ascending)
     bool ok2 = __all_sync(0xffffffffu, *abort == 0);
-    bool polled = false;  // this warp's last readiness poll is behind it
+    // Bounded wait of the whole warp, between polls of tagged words: false
+    // (recording a timeout with the expert) once the budget is spent or the
+    // CTA gave up.
+    unsigned long long poll_t0 = 0;
+    auto poll_more = [&](int it, int u) {
+      if (__any_sync(0xffffffffu, *abort != 0)) return false;
+      if (it == 0) poll_t0 = global_ns();
+      __nanosleep(32);
+      int late = 0;
+      if ((it & 15) == 15) late = global_ns() - poll_t0 > budget ? 1 : 0;
+      if (__shfl_sync(0xffffffffu, late, 0)) {
+        if (lane == 0) {
+          *abort = 1;
+          report_error(a.status, kDevTimeout, 42, u);
+        }
+        return false;
+      }
+      return true;
+    };
     // pass p (base p * nd) gives warp w the experts base + w, base + w + 16, ...
     // below min(nU, base + nd): a warp at or past min(nU, nd) has none at all
     bool cleared = false;
-    if (warp >= min(nU, L.nd)) {
-      polls_done();
-      polled = true;
-      if (clears && nU <= L.nd) {  // one pass: no block barrier ahead that this wait could hold up
-        clear_counters();
-        cleared = true;
-      }
+    if (warp >= min(nU, L.nd) && clears && nU <= L.nd) {  // one pass: no block barrier ahead that this wait could hold up
+      clear_counters();
+      cleared = true;
     }
     for (int base = 0; base < nU; base += L.nd) {
       const uint32_t par = (base / L.nd) & 1u;
@@ -761,73 +803,104 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs
         const int ngd = Iu / kGroup;
         const uint16_t *sd = reinterpret_cast<const uint16_t *>(st + kRowBlock * (Imax / 2));
         const uint16_t *bd = sd + kRowBlock * ngd;
-        // every row block of expert u has published its h
-        ok2 = wait_count(ready + u, static_cast<uint32_t>(Iu / kRowBlock * min(L.ks, 4)), abort, a.status, 42, u,
-                         budget);
-        if (!ok2) break;
-        const bool later_in_pass = u + kSTWarps < min(nU, base + L.nd);
-        const bool later_pass = warp < L.nd && base + L.nd + warp < nU;
-        if (!later_in_pass && !later_pass) {  // the warp's last expert: no more polls
-          polls_done();
-          polled = true;
-        }
         // B fragments: token g's h for this expert (zeros if g is not routed to
-        // it), written by other CTAs of this launch. Where the warp's share of
-        // the token staging area (free once this CTA's gate/up is done) holds
-        // the expert's rows for all T tokens, they are first copied there in
-        // one round trip (cp.async through L2); otherwise read from L2 directly.
+        // it), written as tagged words by other CTAs of this launch and read
+        // through L2 until every word carries this launch's tag. Where the
+        // warp's share of the token staging area (free once this CTA's gate/up
+        // is done) holds the expert's rows for all T tokens, the whole warp
+        // polls them together (one round trip once they are there) and keeps
+        // the values there; otherwise each lane polls its token's words as the
+        // products need them.
         const int jg = (g < T) ? sh.uslot[u][g] : -1;
-        const bool staged = static_cast<size_t>(T) * Iu * 2 <= h_slice_bytes;
-        const __half *hrow;
+        const int cpr = Iu / 4;  // word pairs (16 bytes, four values) per row
+        const bool staged = static_cast<size_t>(T) * Iu * 2 <= h_slice_bytes && T * cpr <= 32 * kPairsPerLane;
+        __half *hw = reinterpret_cast<__half *>(dyn + L.x_off + warp * h_slice_bytes);
         if (staged) {
-          __half *hw = reinterpret_cast<__half *>(dyn + L.x_off + warp * h_slice_bytes);
-          const int cpr = Iu / 8;  // 16-byte chunks per row
-          for (int idx = lane; idx < T * cpr; idx += 32) {
-            const int t = idx / cpr, cc = idx - t * cpr, jt = sh.uslot[u][t];
-            if (jt >= 0)
-              asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(hw + t * Iu + cc * 8)),
-                           "l"(hb + (static_cast<size_t>(t) * (k + 1) + jt) * Imax + cc * 8)
-                           : "memory");
+          const int nch = T * cpr;
+          uint32_t pending = 0;  // bit i: pair lane + 32 i is awaited
+#pragma unroll
+          for (int i = 0; i < kPairsPerLane; ++i) {
+            const int idx = lane + 32 * i;
+            if (idx < nch && sh.uslot[u][idx / cpr] >= 0) pending |= 1u << i;
           }
-          asm volatile("cp.async.wait_all;" ::: "memory");
+          for (int it = 0;; ++it) {
+            ulonglong2 v[kPairsPerLane];
+#pragma unroll
+            for (int i = 0; i < kPairsPerLane; ++i) {
+              const int idx = lane + 32 * i, t = idx / cpr, cc = idx - t * cpr;
+              if ((pending >> i) & 1u)
+                v[i] = ld_tagged2(hb + (static_cast<size_t>(t) * (k + 1) + sh.uslot[u][t]) * (Imax / 2) + 2 * cc);
+            }
+#pragma unroll
+            for (int i = 0; i < kPairsPerLane; ++i) {
+              const int idx = lane + 32 * i, t = idx / cpr, cc = idx - t * cpr;
+              if (((pending >> i) & 1u) && tag_ok(v[i], tag)) {
+                *reinterpret_cast<uint2 *>(hw + t * Iu + 4 * cc) = tagged_values(v[i]);
+                pending &= ~(1u << i);
+              }
+            }
+            if (__all_sync(0xffffffffu, pending == 0)) break;
+            if (!poll_more(it, u)) {
+              ok2 = false;
+              break;
+            }
+          }
+          if (!ok2) break;
           __syncwarp();
-          hrow = hw + (g < T ? g : 0) * Iu;
-        } else {
-          hrow = hb + (static_cast<size_t>(g) * (k + 1) + (jg < 0 ? 0 : jg)) * Imax;
         }
+        const __half *hrow = hw + (g < T ? g : 0) * Iu;  // staged values
+        const uint64_t *trow = hb + (static_cast<size_t>(g) * (k + 1) + (jg < 0 ? 0 : jg)) * (Imax / 2);
         float y[4] = {0.f, 0.f, 0.f, 0.f}, y2[4] = {0.f, 0.f, 0.f, 0.f};  // even / odd words
-        for (int wb = 0; wb < iw; wb += 32) {  // two 16-word blocks per pass: 8 h loads in flight
-          uint4 hv[2][4];
+        for (int w0 = 4 * c; w0 < iw; w0 += 16) {  // 16-word blocks; this thread's words w0 .. w0 + 3
+          uint4 hv[4];
 #pragma unroll
-          for (int b2 = 0; b2 < 2; ++b2)
+          for (int p = 0; p < 4; ++p)
+            hv[p] = (staged && jg >= 0) ? *reinterpret_cast<const uint4 *>(hrow + (w0 + p) * 8) : make_uint4(0, 0, 0, 0);
+          if (!staged) {  // the 8 values of word w0 + p are the tagged pairs 2 (w0 + p) and 2 (w0 + p) + 1
+            uint32_t pending = jg >= 0 ? 0xffu : 0u;
+            for (int it = 0;; ++it) {
+              ulonglong2 v[8];
 #pragma unroll
-            for (int p = 0; p < 4; ++p) {
-              const int w = wb + 16 * b2 + 4 * c + p;
-              hv[b2][p] = make_uint4(0, 0, 0, 0);
-              if (jg >= 0 && w < iw)
-                hv[b2][p] = staged ? *reinterpret_cast<const uint4 *>(hrow + w * 8)
-                                   : __ldcg(reinterpret_cast<const uint4 *>(hrow + w * 8));
+              for (int i = 0; i < 8; ++i)
+                if ((pending >> i) & 1u) v[i] = ld_tagged2(trow + 2 * (2 * (w0 + i / 2) + (i & 1)));
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                if (((pending >> i) & 1u) && tag_ok(v[i], tag)) {
+                  const uint2 q2 = tagged_values(v[i]);
+                  if (i & 1) {
+                    hv[i / 2].z = q2.x;
+                    hv[i / 2].w = q2.y;
+                  } else {
+                    hv[i / 2].x = q2.x;
+                    hv[i / 2].y = q2.y;
+                  }
+                  pending &= ~(1u << i);
+                }
+              }
+              if (__all_sync(0xffffffffu, pending == 0)) break;
+              if (!poll_more(it, u)) {
+                ok2 = false;
+                break;
+              }
             }
+            if (!ok2) break;
+          }
+          const int grp = w0 / 8;
+          const __half2 s0 = bf16_to_half2_bcast(sd[g * ngd + grp]), b0 = bf16_to_half2_bcast(bd[g * ngd + grp]);
+          const __half2 s1 = bf16_to_half2_bcast(sd[(g + 8) * ngd + grp]),
+                        b1 = bf16_to_half2_bcast(bd[(g + 8) * ngd + grp]);
+          const uint4 wd0 = *reinterpret_cast<const uint4 *>(pd + g * iw + w0);
+          const uint4 wd1 = *reinterpret_cast<const uint4 *>(pd + (g + 8) * iw + w0);
+          const uint32_t ad0[4] = {wd0.x, wd0.y, wd0.z, wd0.w}, ad1[4] = {wd1.x, wd1.y, wd1.z, wd1.w};
 #pragma unroll
-          for (int b2 = 0; b2 < 2; ++b2) {
-            if (wb + 16 * b2 >= iw) break;
-            const int w0 = wb + 16 * b2 + 4 * c;
-            const int grp = w0 / 8;
-            const __half2 s0 = bf16_to_half2_bcast(sd[g * ngd + grp]), b0 = bf16_to_half2_bcast(bd[g * ngd + grp]);
-            const __half2 s1 = bf16_to_half2_bcast(sd[(g + 8) * ngd + grp]),
-                          b1 = bf16_to_half2_bcast(bd[(g + 8) * ngd + grp]);
-            const uint4 wd0 = *reinterpret_cast<const uint4 *>(pd + g * iw + w0);
-            const uint4 wd1 = *reinterpret_cast<const uint4 *>(pd + (g + 8) * iw + w0);
-            const uint32_t ad0[4] = {wd0.x, wd0.y, wd0.z, wd0.w}, ad1[4] = {wd1.x, wd1.y, wd1.z, wd1.w};
-#pragma unroll
-            for (int p = 0; p < 4; ++p) {
-              const uint4 d0 = dequant_word(ad0[p], s0, b0), d1 = dequant_word(ad1[p], s1, b1);
-              float(&yy)[4] = (p & 1) ? y2 : y;
-              mma16816(yy, d0.x, d1.x, d0.y, d1.y, hv[b2][p].x, hv[b2][p].y);
-              mma16816(yy, d0.z, d1.z, d0.w, d1.w, hv[b2][p].z, hv[b2][p].w);
-            }
+          for (int p = 0; p < 4; ++p) {
+            const uint4 d0 = dequant_word(ad0[p], s0, b0), d1 = dequant_word(ad1[p], s1, b1);
+            float(&yy)[4] = (p & 1) ? y2 : y;
+            mma16816(yy, d0.x, d1.x, d0.y, d1.y, hv[p].x, hv[p].y);
+            mma16816(yy, d0.z, d1.z, d0.w, d1.w, hv[p].z, hv[p].w);
           }
         }
+        if (!ok2) break;
         // weight each token's column by its routing weight (1 for the shared expert) and 2^(2e)
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -840,7 +913,6 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs
         }
       }
     }
-    if (!polled) polls_done();  // a wait gave up before the last poll
     if (clears && !cleared) clear_counters();
     float *rp = red + static_cast<size_t>(threadIdx.x) * 8;
 #pragma unroll

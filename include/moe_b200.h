@@ -84,8 +84,9 @@ enum {
    * nothing traps. The checks cost a few instructions per work item. */
   MOE_FLAG_DEBUG = 4,
   /* Testing only: the plan's first small-T launch makes one of its bounded
-   * waits run out (row block 0 of the shared expert does not announce that
-   * its SwiGLU output is ready) with a 2 ms budget instead of 2 s; every
+   * waits run out (row block 0 of the shared expert does not store its
+   * SwiGLU output, so its readers never see this launch's tag on it) with a
+   * 2 ms budget instead of 2 s; every
    * other wait of that launch is bounded too and the launch ends normally.
    * moe_status_sync then reports MOE_ERR_DEVICE_TIMEOUT and clears the
    * state, and later calls on the plan run normally. */
@@ -279,24 +280,25 @@ moe_status moe_profile_read(moe_plan_t *plan, moe_stream_t stream, double *ms, i
  * The source pages describe no such call; it exists for callers that
  * cannot call cudaMalloc (code running inside an allocator or memory-pool
  * callback, runtimes that reserve all device memory up front), and so cannot
- * create a plan. Its scratch memory (SwiGLU outputs, the kernel's readiness
- * counters, status word) lives in one static __device__ array of 512 KiB
+ * create a plan. Its scratch memory (SwiGLU outputs, the kernel's counters
+ * and launch tag, status word) lives in one static __device__ array of 512 KiB
  * inside the library, which every GPU that loads the library holds until the
  * process exits; the caller passes only inputs and outputs, as for
  * moe_forward, and gets the same result bit for bit.
  *   Sizes: hidden a multiple of 256 (at most 16384), inter and shared_inter
  *   multiples of 128 (at most 8192), top_k <= min(n_experts, 16),
- *   n_experts <= 256; and the fp16 SwiGLU outputs,
- *   8 * (top_k + 1) * max(inter, shared_inter) * 2 bytes, must fit in
- *   512 KiB - 1280 bytes. Larger layers get MOE_ERR_UNSUPPORTED, T > 8 and
- *   bad sizes MOE_ERR_INVALID_ARG.
+ *   n_experts <= 256; and the SwiGLU outputs (fp16 values stored in pairs
+ *   with a 4-byte launch tag), 8 * (top_k + 1) * max(inter, shared_inter)
+ *   * 4 bytes, must fit in 512 KiB - 1280 bytes. Larger layers get
+ *   MOE_ERR_UNSUPPORTED, T > 8 and bad sizes MOE_ERR_INVALID_ARG.
  *   status_out: optional device pointer to 16 bytes (16-byte aligned) that
  *   receive the device status word of this call ({code, site, detail, 0};
  *   code 0 = OK); a call with T == 0 writes a zero status there.
  * The first call on a device looks up the array's device address (once per
  * device, with that device current; a failed lookup is retried by the next
  * call); make that first call before capturing the stream into a CUDA graph.
- * Each call clears the counters and the status word on the stream and calls
+ * Each call clears the counters and the status word on the stream (the
+ * launch tag is kept, so no call reuses an earlier call's tag) and calls
  * no cudaMalloc, cudaFree or allocating library routine. All calls on one
  * device share that device's copy of the array, so calls that overlap on the
  * GPU (for example on two streams) race: serialise them on one stream.

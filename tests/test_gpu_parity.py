@@ -277,6 +277,29 @@ def test_debug_range_checks_pass_on_valid_runs(case):
     check_output(got, ref, f"debug {case}")
 
 
+@pytest.mark.parametrize("T", [1, 3])
+def test_small_batch_launches_read_only_their_own_swiglu_outputs(T):
+    """The small-batch kernel hands each SwiGLU output between CTAs as a word
+    tagged with its launch. Two inputs alternated on one plan and one layer
+    (T = 1: the readers poll whole rows together; T = 3: each lane polls its
+    own words) give each input its own result, bit for bit on every launch
+    and within tolerance of the oracle: no launch uses words an earlier one
+    left in the scratch."""
+    import dataclasses
+    a = synth.make_layer(T, 2048, 256, 8, 512, 512, seed=611, logit_std=2.0)
+    rng = np.random.default_rng(612)
+    b = dataclasses.replace(a, x=synth.bf16_rne(rng.standard_normal((T, 2048), dtype=np.float32)),
+                            logits=synth.draw_logits(rng, T, 256, 8, 2.0, None))
+    layer = _layer(a)
+    plan = _plan(a)
+    ra, rb = _forward(plan, a, layer), _forward(plan, b, layer)
+    check_output(ra, oracle.moe_forward(a), f"T={T} input a")
+    check_output(rb, oracle.moe_forward(b), f"T={T} input b")
+    for rep in range(3):
+        assert np.array_equal(_forward(plan, a, layer), ra), f"T={T} input a, repeat {rep}"
+        assert np.array_equal(_forward(plan, b, layer), rb), f"T={T} input b, repeat {rep}"
+
+
 def test_bounded_wait_runs_out_and_the_plan_recovers():
     """The test flag makes one wait of the plan's first small-T launch run out
     (row block 0 of the shared expert never announces its output) under a

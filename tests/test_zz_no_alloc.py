@@ -71,7 +71,7 @@ def test_noalloc_rejects_sizes_beyond_its_scratch():
     f = lib.moe_forward_small_t_noalloc
     f.argtypes = [ctypes.c_int] * 6 + [ctypes.c_void_p] * 11
     f.restype = ctypes.c_int
-    # 8 * (16 + 1) * 8192 * 2 bytes of fp16 outputs > 512 KiB
+    # 8 * (16 + 1) * 8192 * 4 bytes of tagged outputs > 512 KiB
     rc = f(1, 2048, 64, 16, 8192, 512, *([None] * 11))
     assert rc == -2 and "512 KiB" in api.moe_last_error()
     rc = f(9, 2048, 256, 8, 512, 512, *([None] * 11))
