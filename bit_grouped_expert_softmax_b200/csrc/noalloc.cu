@@ -6,7 +6,7 @@
 // allocation API is not reachable from the thread that issues work. For them,
 // moe_forward_small_t_noalloc runs the fused small-T kernel (batches of at
 // most 8 tokens) with its scratch memory -- the per-token SwiGLU outputs, the
-// kernel's readiness counters and the device status word -- taken from one
+// kernel's counters and launch tag, and the device status word -- taken from one
 // file-scope __device__ array instead of a plan's workspace. The caller still
 // passes all inputs and outputs.
 //

@@ -631,7 +631,7 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs
   const int rounds = (my_units + units_per_round - 1) / units_per_round;
   const bool slot_used = slot < units_per_round;  // warps of an unused slot only join the barriers
   const int ng = H / kGroup;
-  const int n_pub = min(L.ks, 4);  // publishing warps per unit (readiness count per unit)
+  const int n_pub = min(L.ks, 4);  // warps per unit that reduce its K slices and store its h
   for (int r = 0; r < rounds; ++r) {
     const int q = slot_used ? r * units_per_round + slot : my_units;
     // two accumulator sets per matrix (even and odd words): shorter dependent chains
@@ -698,8 +698,8 @@ __global__ void __launch_bounds__(kSTThreads, 1) small_t_kernel(const SmallTArgs
     __syncthreads();
     const bool live = __all_sync(0xffffffffu, *abort == 0);  // warp-uniform: the block below syncs the warp
     // The unit's first n_pub warps each reduce the C-fragment elements i = kq,
-    // kq + n_pub, ... over the K slices (slice order), store their h and
-    // publish them with their own release increment: a unit counts n_pub.
+    // kq + n_pub, ... over the K slices (slice order) and store their h as
+    // tagged words (the warp is shuffled so that one lane stores each pair).
     if (q < my_units && kq < n_pub && live) {
       // C fragment: rows g (i = 0, 1) and g + 8 (i = 2, 3), token columns 2c, 2c + 1
       for (int i = kq; i < 4; i += n_pub) {
@@ -954,7 +954,7 @@ cudaError_t launch_small_t(const SmallTArgs &a, int num_sms, cudaStream_t s, boo
   cudaError_t err = gemm::ensure_smem_limit(small_t_kernel, static_cast<int>(kStBudget), smem_set);
   if (err != cudaSuccess) return err;
   // cooperative: every CTA resident at once (they wait on one another's
-  // readiness counters); with pdl, also allowed to start while the kernel
+  // SwiGLU outputs); with pdl, also allowed to start while the kernel
   // ahead on the stream finishes
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(small_t_grid(num_sms));
