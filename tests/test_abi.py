@@ -67,3 +67,32 @@ def test_valid_plan_without_gpu_reports_no_device():
     with pytest.raises(api.MoEError) as ei:
         api.moe_plan(16, 256, 16, 2, 128, 128)
     assert ei.value.status == -6
+
+
+@pytest.mark.parametrize("args, rc, fragment", [
+    ((9, 2048, 256, 8, 512, 512), -1, "T must be"),
+    ((1, 384, 16, 2, 128, 128), -1, "hidden"),
+    ((1, 2048, 256, 8, 200, 512), -1, "inter"),
+    ((1, 2048, 256, 8, 512, 100), -1, "inter"),
+    ((1, 2048, 300, 8, 512, 512), -1, "n_experts"),
+    ((1, 2048, 256, 17, 512, 512), -1, "top_k"),
+    # the SwiGLU outputs take 8 * (top_k + 1) * max(I, Is) * 4 bytes (fp16 pairs with
+    # a 4-byte launch tag) of the 512 KiB scratch less its 1280-byte header
+    ((1, 2048, 256, 8, 1920, 512), -2, "512 KiB"),    # 552,960 bytes: too large
+    ((1, 2048, 256, 8, 1792, 512), -1, "pointers"),   # 516,096 bytes: fits, stops at the NULL tensors
+])
+def test_noalloc_rejects_bad_arguments_before_touching_a_gpu(args, rc, fragment):
+    lib = api.load()
+    f = lib.moe_forward_small_t_noalloc
+    f.argtypes = [ctypes.c_int] * 6 + [ctypes.c_void_p] * 11
+    f.restype = ctypes.c_int
+    assert f(*args, *([None] * 11)) == rc
+    assert fragment in api.moe_last_error()
+
+
+def test_noalloc_empty_batch_without_status_does_nothing():
+    lib = api.load()
+    f = lib.moe_forward_small_t_noalloc
+    f.argtypes = [ctypes.c_int] * 6 + [ctypes.c_void_p] * 11
+    f.restype = ctypes.c_int
+    assert f(0, 2048, 256, 8, 512, 512, *([None] * 11)) == 0
